@@ -1,0 +1,425 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix (no GPU).
+
+Each test below would fail for a plausible mistake in the oracle: a dropped term, a wrong
+sign or index, a transposed operand, a wrong scale or an off-by-one in the causal mask.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import mla_inputs as mi
+from oracle import compare, kv_accounting as acc, mla_ref as ref
+from tests.conftest import read_golden, read_table
+
+
+# ----------------------------------------------------------------------------------------
+# Cache arithmetic against the pages' printed values
+# ----------------------------------------------------------------------------------------
+
+def test_cache_table_printed_on_page():
+    for n_heads, kv_heads, mha, gqa, mla in read_table("cache_per_token_table.txt"):
+        assert acc.cache_values_mha(n_heads, 64) == mha
+        assert acc.cache_values_gqa(kv_heads, 64) == gqa
+        assert acc.cache_values_mla(64, 16) == mla
+        assert n_heads == 4 * kv_heads
+
+
+def test_arithmetic_printed_on_pages():
+    g = read_golden("arithmetic_pins.txt")
+    iv = lambda k: int(g[k])  # noqa: E731
+    assert acc.cache_values_mla(iv("glm_kv_rank"), iv("glm_rope_dim")) == iv("glm_cache_values")
+    mha = acc.cache_values_mha(iv("mha_heads"), iv("mha_head_dim"))
+    assert mha == 32768
+    assert round(mha / iv("glm_cache_values")) == iv("glm_saving_x")
+    assert round(100 * acc.reduction_fraction(iv("glm_cache_values"), mha), 1) == float(
+        g["reduction_vs_same_shape_mha_pct"])
+    assert iv("hbm_mha_values") // iv("hbm_latent_values") == iv("hbm_ratio_x")
+    assert acc.cache_values_mha(iv("mha_heads"), iv("mha_head_dim")) == iv("hbm_mha_values")
+    gqa2 = acc.cache_values_gqa(iv("gqa2_kv_heads"), iv("gqa2_head_dim"))
+    assert gqa2 == iv("gqa2_values")
+    mla = acc.cache_values_mla(iv("mla_rank"), iv("mla_rope"))
+    assert mla == iv("mla_values")
+    assert round(gqa2 / mla, 1) == float(g["gqa2_over_mla"])
+    assert acc.gqa_crossover_rank(iv("gqa2_kv_heads"), iv("gqa2_head_dim"), iv("mla_rope")) == iv(
+        "crossover_rank")
+    # at the crossover rank MLA is no longer smaller, one rank below it still is
+    r = iv("crossover_rank")
+    assert acc.cache_values_mla(r, iv("mla_rope")) == gqa2
+    assert acc.cache_values_mla(r - 1, iv("mla_rope")) < gqa2
+    assert acc.cache_values_mha(8, iv("wide_width") // 8) == iv("wide_mha_values")
+    assert iv("train_mha_values") / iv("train_mla_values") == float(g["train_ratio_x"])
+
+
+def test_cache_bytes_formula_matches_code_on_page():
+    # "MLA from scratch in PyTorch", Memory comparison: the page's own function gives
+    # elements * 2 bytes; for MLA at 60 layers, B=1, 4K context, d_c=512 that is 0.25 GB.
+    b = acc.cache_bytes(512, n_layers=60, batch=1, seq=4096)
+    assert b == 512 * 60 * 4096 * 2
+    assert round(b / 1e9, 2) == 0.25
+
+
+def test_decode_work_per_row():
+    # 576-wide bf16 row = 1152 B; 128 heads x 2 x (576 + 512) FLOPs.
+    nbytes, flops = acc.absorbed_decode_work(1, 128, 512, 64)
+    assert nbytes == 1152 and flops == 278528
+    # the naive form's up-projection dominates its FLOPs (what absorption removes)
+    naive = acc.naive_decode_flops(4096, 128, 128, 512)
+    assert naive == 2 * 2 * 4096 * 512 * 128 * 128 + 2 * 128 * 128 * 4096
+
+
+# ----------------------------------------------------------------------------------------
+# Absorption identity, its negative control, and the RoPE counterexample
+# ----------------------------------------------------------------------------------------
+
+def _tiny_inputs(seed=0, L=65, T=1, H=8, dh=32, r=64, dr=16, dtype=np.float64):
+    g = np.random.default_rng([seed, 77])
+    c = g.standard_normal((L, r))
+    kr = g.standard_normal((L, dr))
+    qn = g.standard_normal((T, H, dh))
+    qr = g.standard_normal((T, H, dr))
+    wuk = g.standard_normal((H, dh, r)) / math.sqrt(r)
+    wuv = g.standard_normal((H, dh, r)) / math.sqrt(r)
+    return [x.astype(dtype) for x in (c, kr, qn, qr, wuk, wuv)], 1.0 / math.sqrt(dh + dr)
+
+
+def test_absorption_identity_float64():
+    args, scale = _tiny_inputs()
+    a = ref.naive_decode(*args, scale)
+    b = ref.absorbed_decode(*args, scale)
+    for x, y in zip(a, b):
+        assert np.max(np.abs(x - y)) < 1e-12
+
+
+def test_absorption_identity_float32_at_page_scale():
+    printed = float(read_golden("absorption_identity.txt")["max_abs_diff_printed"])
+    args, scale = _tiny_inputs(dtype=np.float32)
+    a = ref.naive_decode(*args, scale, dtype=np.float32)
+    b = ref.absorbed_decode(*args, scale, dtype=np.float32)
+    d = float(np.max(np.abs(a.o - b.o)))
+    # same order as the page: float32 rounding only, well under 1e-6, not exactly zero
+    assert 0.0 < d < 1e-6
+    assert d < 20 * printed
+
+
+def test_absorption_negative_control_detects_perturbed_wuk():
+    args, scale = _tiny_inputs()
+    c, kr, qn, qr, wuk, wuv = args
+    bad = wuk.copy()
+    bad[3, 5, 7] += 1e-3
+    a = ref.naive_decode(c, kr, qn, qr, bad, wuv, scale)
+    b = ref.absorbed_decode(c, kr, qn, qr, wuk, wuv, scale)
+    assert np.max(np.abs(a.o - b.o)) > 1e-6          # the comparison can fail
+    assert np.max(np.abs(a.o[:, 3] - b.o[:, 3])) > 1e-6
+    others = [h for h in range(8) if h != 3]
+    assert np.max(np.abs(a.o[:, others] - b.o[:, others])) < 1e-12
+
+
+def test_rope_on_reconstructed_key_breaks_absorption():
+    """RoPE applied to the up-projected key makes the score depend on the key's position,
+    so no position-free absorbed matrix can reproduce it; the decoupled key keeps it exact."""
+    g = np.random.default_rng([0, 78])
+    dh, r, base = 16, 32, 10000.0
+    wuk = g.standard_normal((dh, r)) / math.sqrt(r)
+    q = g.standard_normal(dh)
+    c = g.standard_normal(r)
+    pq = 40
+    # same latent c cached at two different positions
+    s_at = [ref.rope_rotate(q, pq, base) @ ref.rope_rotate(wuk @ c, p, base) for p in (3, 17)]
+    assert abs(s_at[0] - s_at[1]) > 1e-3
+    # an absorbed score (A^T q) . c is the same for the two copies of c, whatever A is
+    a = (wuk.T @ ref.rope_rotate(q, pq, base)) @ c
+    assert abs(a - s_at[0]) > 1e-3 or abs(a - s_at[1]) > 1e-3
+    # decoupled: content part unrotated, RoPE only on a separate key -> absorption exact
+    kr = g.standard_normal(8)
+    qr = g.standard_normal(8)
+    for p in (3, 17):
+        naive = q @ (wuk @ c) + ref.rope_rotate(qr, pq, base) @ ref.rope_rotate(kr, p, base)
+        absorbed = (wuk.T @ q) @ c + ref.rope_rotate(qr, pq, base) @ ref.rope_rotate(kr, p, base)
+        assert abs(naive - absorbed) < 1e-12
+
+
+# ----------------------------------------------------------------------------------------
+# Brute force on tiny inputs (pure Python loops, no array arithmetic)
+# ----------------------------------------------------------------------------------------
+
+def _brute_force(c, kr, qn, qr, wuk, wuv, scale):
+    L, r = len(c), len(c[0])
+    T, H, dh = len(qn), len(qn[0]), len(qn[0][0])
+    dr = len(kr[0])
+    dv = len(wuv[0])
+    o = [[[0.0] * dv for _ in range(H)] for _ in range(T)]
+    for t in range(T):
+        n = L - T + 1 + t
+        for h in range(H):
+            s = []
+            for l in range(n):
+                k = [sum(wuk[h][i][j] * c[l][j] for j in range(r)) for i in range(dh)]
+                dot = sum(qn[t][h][i] * k[i] for i in range(dh))
+                dot += sum(qr[t][h][i] * kr[l][i] for i in range(dr))
+                s.append(dot * scale)
+            m = max(s)
+            e = [math.exp(x - m) for x in s]
+            z = sum(e)
+            for i in range(dv):
+                v = [sum(wuv[h][i][j] * c[l][j] for j in range(r)) for l in range(n)]
+                o[t][h][i] = sum(e[l] / z * v[l] for l in range(n))
+    return np.array(o)
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_bruteforce_small(T):
+    args, scale = _tiny_inputs(L=7, T=T, H=3, dh=4, r=6, dr=4)
+    bf = _brute_force(*[a.tolist() for a in args], scale)
+    a = ref.naive_decode(*args, scale)
+    b = ref.absorbed_decode(*args, scale)
+    assert np.max(np.abs(a.o - bf)) < 1e-12
+    assert np.max(np.abs(b.o - bf)) < 1e-12
+
+
+def test_causal_mask_is_not_off_by_one():
+    args, scale = _tiny_inputs(L=9, T=3, H=2, dh=4, r=6, dr=4)
+    c, kr, qn, qr, wuk, wuv = args
+    full = ref.naive_decode(*args, scale)
+    # query t of a T-token step equals a 1-token step over the first L - T + t + 1 rows
+    for t in range(3):
+        n = 9 - 3 + t + 1
+        one = ref.naive_decode(c[:n], kr[:n], qn[t:t + 1], qr[t:t + 1], wuk, wuv, scale)
+        assert np.max(np.abs(one.o[0] - full.o[t])) < 1e-12
+        assert np.max(np.abs(one.lse[0] - full.lse[t])) < 1e-12
+
+
+# ----------------------------------------------------------------------------------------
+# Special cases that reduce to a closed form or a library routine
+# ----------------------------------------------------------------------------------------
+
+def test_single_row_returns_value_of_that_row():
+    args, scale = _tiny_inputs(L=1)
+    c, kr, qn, qr, wuk, wuv = args
+    out = ref.naive_decode(*args, scale)
+    for h in range(wuv.shape[0]):
+        assert np.max(np.abs(out.o[0, h] - wuv[h] @ c[0])) < 1e-14
+    assert np.max(np.abs(out.o_lat[0] - c[0])) < 1e-14
+
+
+def test_identical_rows_make_output_query_independent():
+    args, scale = _tiny_inputs(L=10)
+    c, kr, qn, qr, wuk, wuv = args
+    c[:] = c[0]
+    kr[:] = kr[0]
+    out = ref.naive_decode(c, kr, qn, qr, wuk, wuv, scale)
+    out2 = ref.naive_decode(c, kr, -3.0 * qn, qr + 1.0, wuk, wuv, scale)
+    for h in range(wuv.shape[0]):
+        assert np.max(np.abs(out.o[0, h] - wuv[h] @ c[0])) < 1e-12
+    assert np.max(np.abs(out.o - out2.o)) < 1e-12
+
+
+def test_identity_weights_reduce_to_library_sdpa():
+    g = np.random.default_rng([0, 79])
+    L, r = 12, 16
+    c = g.standard_normal((L, r))
+    q = g.standard_normal((1, 1, r))
+    eye = np.eye(r)[None]
+    out = ref.naive_decode(c, np.zeros((L, 0)), q, np.zeros((1, 1, 0)), eye, eye, 1.0 / math.sqrt(r))
+    t = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q[0][None]), torch.from_numpy(c[None]), torch.from_numpy(c[None]))
+    assert np.max(np.abs(out.o[0, 0] - t.numpy()[0, 0])) < 1e-12
+
+
+def test_softmax_rows_sum_to_one_and_masked_entries_are_zero():
+    g = np.random.default_rng([0, 80])
+    s = g.standard_normal((5, 17)) * 10
+    s[:, 11:] = -np.inf
+    p = ref.softmax(s)
+    assert np.max(np.abs(p.sum(-1) - 1.0)) < 1e-12
+    assert np.all(p[:, 11:] == 0.0)
+    assert np.max(np.abs(ref.logsumexp(s) - np.log(np.exp(s).sum(-1)))) < 1e-12
+
+
+def test_latent_outputs_and_lse_consistent():
+    args, scale = _tiny_inputs(L=20, T=2)
+    out = ref.naive_decode(*args, scale)
+    c, kr, qn, qr, wuk, wuv = args
+    Q = np.concatenate([ref.absorb_query(qn, wuk), qr], axis=-1)
+    lat = ref.latent_attention(Q, np.concatenate([c, kr], axis=1), c.shape[1], scale, T=2)
+    assert np.max(np.abs(lat.o_lat - out.o_lat)) < 1e-12
+    assert np.max(np.abs(lat.lse - out.lse)) < 1e-12
+    assert np.max(np.abs(ref.output_ref(lat.o_lat, wuv) - out.o)) < 1e-12
+
+
+def test_combine_of_disjoint_ranges_equals_whole():
+    g = np.random.default_rng([0, 81])
+    L, H, r, dr = 50, 4, 8, 4
+    rows = g.standard_normal((L, r + dr))
+    Q = g.standard_normal((1, H, r + dr)) * 2
+    whole = ref.latent_attention(Q, rows, r, 0.3, T=1)
+    cuts = [0, 7, 8, 31, 50]
+    parts = [ref.latent_attention(Q, rows[a:b], r, 0.3, T=1) for a, b in zip(cuts[:-1], cuts[1:])]
+    o, L_ = ref.combine_ref([p.o_lat for p in parts], [p.lse for p in parts])
+    assert np.max(np.abs(o - whole.o_lat)) < 1e-12
+    assert np.max(np.abs(L_ - whole.lse)) < 1e-12
+    # one part: the combine is the identity
+    o1, l1 = ref.combine_ref([whole.o_lat], [whole.lse])
+    assert np.max(np.abs(o1 - whole.o_lat)) == 0 and np.max(np.abs(l1 - whole.lse)) == 0
+
+
+# ----------------------------------------------------------------------------------------
+# RoPE, RMSNorm, bf16 rounding, projections
+# ----------------------------------------------------------------------------------------
+
+def test_rope_matches_complex_rotation_and_properties():
+    g = np.random.default_rng([0, 82])
+    d, base = 16, 10000.0
+    x = g.standard_normal((5, d))
+    pos = np.array([0, 1, 7, 100, 32767])
+    y = ref.rope_rotate(x, pos, base)
+    # complex form: (x0 + i x1) * exp(i * pos * base^(-2k/d))
+    z = (x[:, 0::2] + 1j * x[:, 1::2]) * np.exp(
+        1j * pos[:, None] * base ** (-2.0 * np.arange(d // 2) / d))
+    assert np.max(np.abs(y[:, 0::2] - z.real)) < 1e-12
+    assert np.max(np.abs(y[:, 1::2] - z.imag)) < 1e-12
+    assert np.max(np.abs(np.linalg.norm(y, axis=1) - np.linalg.norm(x, axis=1))) < 1e-12
+    assert np.max(np.abs(y[0] - x[0])) == 0.0                 # position 0 is the identity
+    q, k = x[1], x[2]
+    # relative position: (R_p q).(R_p' k) depends only on p - p'
+    a = ref.rope_rotate(q, 50, base) @ ref.rope_rotate(k, 20, base)
+    b = ref.rope_rotate(q, 1030, base) @ ref.rope_rotate(k, 1000, base)
+    assert abs(a - b) < 1e-10
+    assert abs(a - ref.rope_rotate(q, 30, base) @ k) < 1e-10
+    # the first pair turns fastest: theta_0 = 1, theta_last = base^(-(d-2)/d)
+    th = ref.rope_inv_freq(d, base)
+    assert th[0] == 1.0 and abs(th[-1] - base ** (-(d - 2) / d)) < 1e-18
+
+
+def test_rmsnorm_closed_form_and_library():
+    g = np.random.default_rng([0, 83])
+    x = g.standard_normal((6, 64)) * 3
+    eps = 1e-6
+    y = ref.rms_norm(x, np.ones(64), eps)
+    ms = np.mean(x * x, axis=1)
+    assert np.max(np.abs(np.mean(y * y, axis=1) - ms / (ms + eps))) < 1e-12
+    gam = 1 + 0.1 * g.standard_normal(64)
+    lib = torch.nn.functional.rms_norm(torch.from_numpy(x), (64,), torch.from_numpy(gam), eps)
+    assert np.max(np.abs(ref.rms_norm(x, gam, eps) - lib.numpy())) < 1e-12
+
+
+def test_round_bf16_matches_library_conversion():
+    g = np.random.default_rng([0, 84])
+    vals = [g.standard_normal(20000).astype(np.float32),
+            (g.standard_normal(2000) * 1e-39).astype(np.float32),      # subnormals
+            (g.standard_normal(2000) * 1e38).astype(np.float32),       # near overflow
+            np.array([0.0, -0.0, 1.0, 1.00390625, 1.01171875, 3.3895314e38, -3.3961814e38],
+                     dtype=np.float32)]
+    # exact ties: 1 + 2^-8 (tie, rounds to 1) and 1 + 3*2^-8 (tie, rounds up to 1 + 2^-6)
+    ties = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8)], dtype=np.float32)
+    for v in vals + [ties]:
+        lib = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+        mine = ref.round_bf16(v.astype(np.float64))
+        assert np.array_equal(mine, lib, equal_nan=True), v[mine != lib][:5]
+    assert ref.round_bf16(np.array([1 + 2 ** -8]))[0] == 1.0
+    assert ref.round_bf16(np.array([1 + 3 * 2 ** -8]))[0] == 1 + 2 ** -6
+
+
+def test_project_layer_matches_library_linear():
+    w = mi.WORKLOADS["small_fp32"]
+    d = mi.layer_draw(mi.scaled(w, batch=2, cached=5))
+    p = ref.project_layer(d.x, w.num_heads, w.head_dim, w.rope_dim, d.w_dkv, d.w_kr, d.w_qr,
+                          w_dq=d.w_dq, w_uq=d.w_uq, gamma_q=d.gamma_q, eps=w.rms_eps)
+    F = torch.nn.functional
+    x = torch.from_numpy(d.x)
+    cq = F.rms_norm(F.linear(x, torch.from_numpy(d.w_dq)), (w.q_rank,), eps=w.rms_eps)
+    q = F.linear(cq, torch.from_numpy(d.w_uq)).reshape(2, -1, w.num_heads, w.head_dim)
+    assert np.max(np.abs(p.q_nope - q.numpy())) < 1e-12
+    assert np.max(np.abs(p.ckv_raw - F.linear(x, torch.from_numpy(d.w_dkv)).numpy())) < 1e-12
+    assert np.max(np.abs(p.krope_raw - F.linear(x, torch.from_numpy(d.w_kr)).numpy())) < 1e-12
+
+
+# ----------------------------------------------------------------------------------------
+# Paged placement (integer work: exact)
+# ----------------------------------------------------------------------------------------
+
+def test_paged_placement_bruteforce_and_invalid_entries():
+    g = np.random.default_rng([0, 85])
+    B, maxb, bs, nb = 3, 4, 5, 9
+    table = g.permutation(nb)[: B * maxb - 3].tolist() + [-1, 99, 4]
+    table = np.array(table, dtype=np.int32).reshape(B, maxb)
+    seq = g.integers(0, B, 200)
+    pos = g.integers(-2, maxb * bs + 3, 200)
+    pl = ref.paged_placement(seq, pos, table, bs, nb)
+    for i in range(200):
+        b, p = int(seq[i]), int(pos[i])
+        ok = 0 <= p < maxb * bs and 0 <= table[b][p // bs] < nb
+        assert bool(pl.valid[i]) == ok
+        if ok:
+            assert pl.block[i] == table[b][p // bs] and pl.slot[i] == p % bs
+
+
+def test_append_grows_cache_like_the_shape_trace():
+    g = read_golden("shape_trace.txt")
+    B, S, r = int(g["batch"]), int(g["prefill"]), int(g["latent"])
+    bs = 4
+    nblk = (S + 1 + bs - 1) // bs
+    table = np.arange(B * nblk, dtype=np.int32).reshape(B, nblk)
+    pool = np.full((B * nblk, bs, r + 2), np.nan)
+    rng = np.random.default_rng([0, 86])
+    seq = np.repeat(np.arange(B), S)
+    pos = np.tile(np.arange(S), B)
+    ref.append_ref(pool, rng.standard_normal((B * S, r)), rng.standard_normal((B * S, 2)),
+                   np.ones(r), seq, pos, table, bs, 1e-6, 1e4, False)
+    filled = lambda b: sum(np.isfinite(pool[table[b], :, 0]).ravel())  # noqa: E731
+    assert [B, filled(0), r] == [int(v) for v in g["after_prefill"]]
+    ref.append_ref(pool, rng.standard_normal((B, r)), rng.standard_normal((B, 2)), np.ones(r),
+                   np.arange(B), np.full(B, S), table, bs, 1e-6, 1e4, False)
+    assert [B, filled(0), r] == [int(v) for v in g["after_one_step"]]
+    assert filled(1) == S + 1
+
+
+# ----------------------------------------------------------------------------------------
+# The tolerance harness itself must be able to fail
+# ----------------------------------------------------------------------------------------
+
+def _small_decode(dtype="bf16"):
+    w = mi.scaled(mi.WORKLOADS["small_bf16"], batch=1, cached=200)
+    rows = int(mi.total_rows(w)[0])
+    d = mi.sequence_draw(w, 0, rows)
+    wuk, wuv = mi.up_projection_weights(w)
+    return w, d, wuk, wuv, ref.decode_sequence_from_raw(
+        d.ckv_raw, d.krope_raw, d.q_nope, d.q_rope_raw, wuk, wuv, np.ones(w.kv_rank),
+        w.softmax_scale, w.rms_eps, w.rope_base, store_bf16=True)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_tolerance_negative_controls(dtype):
+    w, d, wuk, wuv, out = _small_decode()
+    o = out.o[0]
+    ok, _ = compare.within(o, o, dtype)
+    assert ok
+    assert not compare.within(np.zeros_like(o), o, dtype)[0]
+    swapped = o.copy()
+    swapped[[0, 1]] = swapped[[1, 0]]
+    assert not compare.within(swapped, o, dtype)[0]
+    # a one-token shift of the query position changes the output beyond tolerance
+    rows = d.ckv_raw.shape[0]
+    c = ref.cache_rows(d.ckv_raw, d.krope_raw, np.ones(w.kv_rank), np.arange(rows), w.rms_eps,
+                       w.rope_base, True)
+    qr = ref.rope_rotate(d.q_rope_raw.astype(np.float64), np.array([[rows - 2]]), w.rope_base)
+    shifted = ref.naive_decode(c[:, :w.kv_rank], c[:, w.kv_rank:], d.q_nope, qr, wuk, wuv,
+                               w.softmax_scale)
+    assert not compare.within(shifted.o[0], o, dtype)[0]
+
+
+def test_needle_makes_attention_peaky():
+    w = mi.scaled(mi.WORKLOADS["small_bf16"], batch=1, cached=300)
+    rows = int(mi.total_rows(w)[0])
+    d = mi.sequence_draw(w, 0, rows)
+    j = mi.plant_needle(w, d)
+    wuk, wuv = mi.up_projection_weights(w)
+    c = ref.cache_rows(d.ckv_raw, d.krope_raw, np.ones(w.kv_rank), np.arange(rows), w.rms_eps,
+                       w.rope_base, True)
+    qr = ref.rope_rotate(d.q_rope_raw.astype(np.float64), np.array([[rows - 1]]), w.rope_base)
+    Q = np.concatenate([ref.absorb_query(d.q_nope, wuk), qr], axis=-1)
+    s = np.einsum("thd,ld->thl", Q, c) * w.softmax_scale
+    p = ref.softmax(s)
+    assert p[0, :, j].max() > 0.5
+    assert np.argmax(p[0].max(axis=1)) is not None
