@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Throughput of one MLA absorbed decode step on B200, as one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dsv2] [--impl ours|reference]
+
+A step is the whole hot path over one batch: mla_absorb_query, mla_append_latent, mla_decode
+(plan, attention, combine) and mla_output, on synthetic inputs of the DeepSeek-V2 attention
+shape (H=128, d_h=128, r=512, d_r=64, B=64 sequences of S=8192 cached rows, paged 64-row
+blocks with a permuted table). Every rank owns its own batch (weak scaling, no collective on
+the data path); ``value`` is the tokens decoded by all ranks divided by the slowest rank's
+device time. ``--impl reference`` times the CPU float64 oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA absorbed decode: cache TB/s (frac of HBM/MMA roofline), tokens/s, B=64 S=8k"
+REF_BUDGET_S = 150.0  # whole --impl reference run
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="dsv2")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-kernel", default="auto", choices=["auto", "simt", "tensor"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def workload_desc(w):
+    return (f"{w.name}: H={w.num_heads} d_h={w.head_dim} r={w.kv_rank} d_r={w.rope_dim} "
+            f"B={w.batch} S={w.cached if not w.ragged_max else 'U[1,%d]' % w.ragged_max} "
+            f"T={w.new_tokens} {w.dtype} paged {w.block_size}-row blocks")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------------------
+# clocks sampled by nvidia-smi while the timed region runs
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.samples = []
+        self.proc = None
+        self.gpu_id = gpu_id
+        self.window = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [(t, s) for t, s in self.samples if t0 <= t <= t1]
+        window = "timed region"
+        if not rows and self.samples:
+            mid = 0.5 * (t0 + t1)
+            rows = sorted(self.samples, key=lambda x: abs(x[0] - mid))[:3]
+            window = "nearest samples to a timed region shorter than the sampling period"
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, s in rows:
+            parts = [p.strip() for p in s.split(",")]
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm), "window": window}
+
+
+# ---------------------------------------------------------------------------------------
+# the CPU oracle on a bounded sample (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------------------
+def oracle_sample(w, heads: int, seed: int = 0):
+    """Inputs of sequence 0 restricted to the first ``heads`` heads, as the GPU stores them."""
+    import numpy as np
+
+    import mla_inputs as mi
+
+    rows = int(mi.total_rows(w, seed)[0])
+    d = mi.sequence_draw(w, 0, rows, seed)
+    wuk, wuv = mi.up_projection_weights(w, seed)
+    st = lambda x: mi.storage_round(w, x)  # noqa: E731
+    return (st(d.ckv_raw), st(d.krope_raw), st(d.q_nope)[:, :heads], st(d.q_rope_raw)[:, :heads],
+            st(wuk)[:heads], st(wuv)[:heads], np.ones(w.kv_rank, np.float32))
+
+
+def oracle_run(w, inputs):
+    from oracle import mla_ref
+
+    ckv, kr, qn, qr, wuk, wuv, gamma = inputs
+    return mla_ref.decode_sequence_from_raw(ckv, kr, qn, qr, wuk, wuv, gamma, w.softmax_scale,
+                                            w.rms_eps, w.rope_base, store_bf16=(w.dtype == "bf16"),
+                                            form="naive")
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, budget_s: float = 20.0):
+    """Naive float64 oracle on whole heads of one sequence, as many heads as fit the budget."""
+    one = oracle_sample(w, 1)
+    t0 = time.perf_counter()
+    oracle_run(w, one)
+    t_head = time.perf_counter() - t0
+    heads = int(max(1, min(w.num_heads, budget_s / max(t_head, 1e-6))))
+    inp = oracle_sample(w, heads)
+    t0 = time.perf_counter()
+    oracle_run(w, inp)
+    dt = time.perf_counter() - t0
+    tokens = w.new_tokens * heads / w.num_heads
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"naive float64 oracle (K and V rebuilt per head), sequence 0 of {w.name}: "
+                       f"{heads} of "
+                       f"{w.num_heads} heads over {int(inp[0].shape[0])} rows, {dt:.1f} s; "
+                       f"value = query tokens (heads/{w.num_heads} per token) per second")}
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    per_step = REF_BUDGET_S / max(1, args.steps + args.warmup)
+    one = oracle_sample(w, 1)
+    t0 = time.perf_counter()
+    oracle_run(w, one)
+    t_head = time.perf_counter() - t0
+    heads = int(max(1, min(w.num_heads, per_step / max(t_head, 1e-6))))
+    inp = oracle_sample(w, heads)
+    for _ in range(args.warmup):
+        oracle_run(w, inp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_run(w, inp)
+    dt = time.perf_counter() - t0
+    tokens = args.steps * w.new_tokens * heads / w.num_heads
+    value = tokens / dt
+    sample = (f"naive float64 oracle on {heads} of {w.num_heads} heads of one "
+              f"{int(inp[0].shape[0])}-row sequence per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(w), "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import mla_latent_kv_44_b200 as mla
+    from mla_latent_kv_44_b200.step import DecodeState
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    kernel = {"auto": mla.DECODE_AUTO, "simt": mla.DECODE_SIMT,
+              "tensor": mla.DECODE_TENSOR}[args.decode_kernel]
+    st = DecodeState(w, seed=rank, device=str(dev), decode_kernel=kernel)
+    stream = torch.cuda.Stream(device=dev)
+    B, T = w.batch, w.new_tokens
+    tokens_per_step = B * T
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- warm-up ----
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            st.step(stream)
+    stream.synchronize()
+    if int(st.dev_err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(st.dev_err.item())}")
+
+    # ---- timed region: K steps, per-stage events on the launching stream ----
+    names = ["absorb", "append", "plan", "attend", "combine", "output"]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+          for _ in range(args.steps)]
+    clock = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid)
+                         if hasattr(torch.cuda.get_device_properties(dev), "uuid") else str(local))
+    if rank == 0:
+        clock.start()
+        time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    with torch.cuda.stream(stream):
+        for k in range(args.steps):
+            e = ev[k]
+            e[0].record(stream)
+            st.absorb(stream)
+            e[1].record(stream)
+            st.append(stream)
+            e[2].record(stream)
+            st.attend(stream, mla.STAGE_PLAN)
+            e[3].record(stream)
+            st.attend(stream, mla.STAGE_ATTEND)
+            e[4].record(stream)
+            st.attend(stream, mla.STAGE_COMBINE)
+            e[5].record(stream)
+            st.project(stream)
+            e[6].record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier()
+    elapsed_ms = ev[0][0].elapsed_time(ev[-1][-1])
+    stage_ms = {n: sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)) / args.steps
+                for i, n in enumerate(names)}
+    if int(st.dev_err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(st.dev_err.item())}")
+
+    # ---- e2e through host buffers: H2D of the step's inputs, the four calls, D2H of o ----
+    host_in = [t.cpu().pin_memory() for t in (st.q_nope, st.q_rope, st.ckv_new, st.krope_new,
+                                              st.seq_new, st.pos_new, st.seq_lens)]
+    dev_in = [st.q_nope, st.q_rope, st.ckv_new, st.krope_new, st.seq_new, st.pos_new, st.seq_lens]
+    host_out = torch.empty(st.o.shape, dtype=st.o.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = min(args.steps, 200)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            for hsrc, ddst in zip(host_in, dev_in):
+                ddst.copy_(hsrc, non_blocking=True)
+            st.step(stream)
+            host_out.copy_(st.o, non_blocking=True)
+    stream.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            for hsrc, ddst in zip(host_in, dev_in):
+                ddst.copy_(hsrc, non_blocking=True)
+            st.step(stream)
+            host_out.copy_(st.o, non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    barrier()
+
+    # ---- max over ranks ----
+    t = torch.tensor([elapsed_ms, e2e_ms, stage_ms["attend"]], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms, attend_ms = (float(x) for x in t.tolist())
+    if rank == 0:
+        clock.stop()
+    clocks = clock.summary(t_wall0, t_wall1) if rank == 0 else None
+    del st
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    import mla_inputs as mi
+
+    rows = mi.total_rows(w, 0)
+    attended = int(sum(int(n) - T + 1 + t_ for n in rows for t_ in range(T)))
+    row_bytes = w.row_width * 2
+    flops_row = w.num_heads * 2 * (w.row_width + w.kv_rank)
+    attend_bytes = attended * row_bytes
+    attend_flops = attended * flops_row
+    hbm, tc_burst, tc_sust, peak_src = load_peaks()
+    attend_s = attend_ms * 1e-3
+    gbs = attend_bytes / attend_s / 1e9
+    tflops = attend_flops / attend_s / 1e12
+    bound = "hbm" if attend_bytes / (hbm * 1e9) >= attend_flops / (tc_burst * 1e12) else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}
+    else:
+        roof = {"bound": "tensor", "achieved": tflops, "peak": tc_burst, "unit": "TFLOP/s",
+                "frac": tflops / tc_burst}
+    roof.update({"traffic": None, "kernel": "mla attention (split-KV main)",
+                 "algorithmic_bytes_per_launch": attend_bytes,
+                 "algorithmic_flops_per_launch": attend_flops,
+                 "avg_launch_us": attend_ms * 1e3, "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"
+                 if peak_src == "measured" else "fallback",
+                 "tensor_view": {"achieved_tflops": tflops, "peak": tc_burst,
+                                 "frac": tflops / tc_burst}})
+    ms_per_step = elapsed_ms / args.steps
+    value = tokens_per_step * world * args.steps / (elapsed_ms * 1e-3)
+    e2e_value = tokens_per_step * world * e2e_steps / (e2e_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) projections, N(0,1/r) weights; per-rank seed)",
+        "config": {"workload": workload_desc(w), "batch_per_gpu": B, "global_batch": B * world,
+                   "seq_len": int(rows.max()) - T, "new_tokens": T,
+                   "parallelism": f"dp{world} (sequence-sharded replicas, no collective)",
+                   "l2": f"inputs larger than L2: {attend_bytes / 1e9:.2f} GB of cache per step",
+                   "decode_kernel": args.decode_kernel},
+        "roofline": roof,
+        "cache_tbs": gbs / 1e3,
+        "attend_tflops": tflops,
+        "stages_us": {k: v * 1e3 for k, v in stage_ms.items()},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    import mla_inputs as mi
+
+    w = mi.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

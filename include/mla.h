@@ -1,0 +1,175 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) library for DeepSeek-V2 Multi-head Latent Attention
+ * decode in absorbed form over a paged latent KV cache.
+ *
+ * Sources for the operations (page title, then section or figure):
+ *   [A] "DeepSeek MLA, Built From the Paper", 3 Matrix absorption:
+ *       q^T (W_UK c_kv) = (W_UK^T q)^T c_kv -- W_UK folds into the query; no key is rebuilt.
+ *   [B] "MLA from scratch in PyTorch", The MLAAttention module / KV cache management during
+ *       decode / Absorbing projections / What's not in this implementation (paged cache).
+ *   [C] "Build a DeepSeek Model from Scratch", ch. 3 figures: the score is the sum of a
+ *       content score and a position score; the output rearrangement applies W_UV after the
+ *       weighted sum; the new latent is appended to the cache.
+ *   [D] "Multi-head latent attention", Compress keys and values into one latent: each token
+ *       caches c_t (width r) and one RoPE key k_rope_t (width d_r) shared by all heads.
+ *
+ * Conventions shared by every call:
+ *   - Every data pointer is DEVICE memory owned by the caller; the library allocates nothing,
+ *     keeps no state between calls (apart from a per-device SM-count cache) and never frees.
+ *   - Every call only enqueues work on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream) and returns; nothing is synchronised.
+ *   - Tensors are row-major and contiguous. "dtype" tensors are float32 or bfloat16 as
+ *     mla_config.dtype says; out_latent and lse are always float32; gamma is float32.
+ *   - Argument and shape errors return synchronously with no launch. Data-dependent errors
+ *     found on the device (a block id outside the pool, a position outside the block table,
+ *     an impossible sequence length, a bounded wait that gave up) set bits in *dev_err
+ *     (atomicOr) and skip the affected work; kernels never trap. The caller clears *dev_err.
+ *   - Empty work (n_tokens == 0, batch == 0) returns MLA_OK without launching.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad config value          */
+  MLA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. tensor-core decode shape)   */
+  MLA_ERR_CUDA = 3,        /* a launch or runtime call failed                             */
+  MLA_ERR_WORKSPACE = 4    /* workspace pointer misaligned or smaller than required       */
+} mla_status;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
+
+/* Which attention kernel mla_decode uses. AUTO picks the tcgen05 tensor-core kernel for
+ * bf16 at H=128, r=512, d_r=64, block_size=64, and the CUDA-core kernel otherwise. */
+typedef enum { MLA_DECODE_AUTO = 0, MLA_DECODE_SIMT = 1, MLA_DECODE_TENSOR = 2 } mla_decode_kernel;
+
+typedef struct {
+  int32_t num_heads;     /* H                                                    */
+  int32_t head_dim;      /* d_h: width of q_nope and of each head's content key  */
+  int32_t head_dim_v;    /* d_v: width of each head's value / output             */
+  int32_t kv_rank;       /* r: width of the cached latent c_kv (multiple of 32)  */
+  int32_t rope_dim;      /* d_r: width of the decoupled RoPE key (even, may be 0) */
+  int32_t block_size;    /* tokens per cache block                               */
+  float rope_base;       /* RoPE base (10000)                                    */
+  float rms_eps;         /* RMSNorm epsilon (1e-6)                               */
+  float softmax_scale;   /* multiplies Q . row before the softmax (1/sqrt(d_h+d_r)) */
+  int32_t dtype;         /* mla_dtype of activations, weights and the cache      */
+  int32_t decode_kernel; /* mla_decode_kernel                                    */
+} mla_config;
+
+/* Bits of the device error word. */
+#define MLA_DEV_OOB_BLOCK 1u    /* block_table entry outside [0, num_blocks)                  */
+#define MLA_DEV_OOB_POS 2u      /* sequence index or position outside the block table         */
+#define MLA_DEV_WAIT_TIMEOUT 4u /* a bounded wait inside a kernel gave up; results invalid    */
+#define MLA_DEV_BAD_LENGTH 8u   /* seq_lens[b] < q_per_seq or > max_blocks * block_size      */
+
+/* Rows of the packed absorbed query and of the cache: r + d_r values. */
+
+/*
+ * mla_absorb_query -- [A], [C], [D].
+ *   Q[n, h, 0:r]      = W_UK[h]^T q_nope[n, h]          (fp32 accumulation)
+ *   Q[n, h, r:r+d_r]  = RoPE(q_rope[n, h], pos[n])      (adjacent pairs (2i, 2i+1) rotated by
+ *                                                        pos * rope_base^(-2i/d_r))
+ * q_nope (n_tokens, H, d_h) dtype; q_rope (n_tokens, H, d_r) dtype, un-rotated;
+ * pos (n_tokens) int32 >= 0; w_uk (H, d_h, r) dtype -- the nn.Linear(r, H*d_h) weight,
+ * rows h*d_h .. (h+1)*d_h-1 for head h, i.e. the same memory without a transpose;
+ * q_out (n_tokens, H, r + d_r) dtype, rounded to nearest even when bf16.
+ */
+MLA_API mla_status mla_absorb_query(const mla_config* cfg, const void* q_nope, const void* q_rope,
+                            const int32_t* pos, const void* w_uk, void* q_out, int32_t n_tokens,
+                            void* stream);
+
+/*
+ * mla_append_latent -- [B] (norm_kv before caching; paged cache), [C] (append), [D] (row
+ * layout [c_kv || k_rope]).
+ *   row = [ RMSNorm(ckv_raw[n]) * gamma || RoPE(krope_raw[n], pos[n]) ]  (fp32 math, stored in
+ *   dtype, bf16 rounded to nearest even), written to
+ *   pool[block_table[seq_idx[n] * max_blocks + pos[n] / block_size]][pos[n] % block_size][:].
+ * ckv_raw (n_tokens, r) dtype; krope_raw (n_tokens, d_r) dtype; gamma (r) float32;
+ * seq_idx, pos (n_tokens) int32; block_table (batch, max_blocks) int32;
+ * pool (num_blocks, block_size, r + d_r) dtype. A row whose sequence index or position is
+ * outside the table sets MLA_DEV_OOB_POS, one whose block id is outside the pool sets
+ * MLA_DEV_OOB_BLOCK; neither is written. No other pool byte is touched.
+ */
+MLA_API mla_status mla_append_latent(const mla_config* cfg, const void* ckv_raw, const void* krope_raw,
+                             const float* gamma, const int32_t* seq_idx, const int32_t* pos,
+                             const int32_t* block_table, int32_t batch, int32_t max_blocks,
+                             void* pool, int32_t num_blocks, int32_t n_tokens, uint32_t* dev_err,
+                             void* stream);
+
+/*
+ * Workspace of mla_decode in bytes for this configuration and batch shape (0 when the
+ * configuration is invalid). The workspace holds the split-KV schedule and the partial
+ * outputs of sequences split across work ranges; it must be 256-byte aligned.
+ */
+MLA_API size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t q_per_seq);
+
+/*
+ * mla_decode -- split-KV flash decoding in absorbed form ([A], [B] Absorbing projections:
+ * attend directly to latents; [C] score = content + position).
+ * For sequence b, query token t (bt = b * q_per_seq + t) and head h, with
+ * L = seq_lens[b] - q_per_seq + 1 + t rows attended (rows 0 .. L-1: causal among the new
+ * tokens, each new token sees itself):
+ *   s_j = softmax_scale * Q[bt, h, :] . row_j,   p = softmax(s),
+ *   out_latent[bt, h, :] = sum_j p_j row_j[0:r],  lse[bt, h] = log(sum_j exp(s_j)).
+ * q (batch * q_per_seq, H, r + d_r) dtype; pool and block_table as in mla_append_latent;
+ * seq_lens (batch) int32: rows valid after this step's append (callers advance it by
+ * q_per_seq before the call); out_latent (batch * q_per_seq, H, r) float32;
+ * lse (batch * q_per_seq, H) float32 or NULL. Runs three stages on `stream`: a one-CTA
+ * planner that cuts all (sequence, token) row ranges into equal 64-row chunks of work, the
+ * attention kernel, and a log-sum-exp combine of sequences that were split. A length outside
+ * [1, max_blocks * block_size] sets MLA_DEV_BAD_LENGTH and that row's output is 0 (lse -inf).
+ * Deterministic: the same inputs give the same bits.
+ */
+MLA_API mla_status mla_decode(const mla_config* cfg, const void* q, const void* pool,
+                      const int32_t* block_table, int32_t max_blocks, int32_t num_blocks,
+                      const int32_t* seq_lens, int32_t batch, int32_t q_per_seq, void* workspace,
+                      size_t workspace_bytes, float* out_latent, float* lse, uint32_t* dev_err,
+                      void* stream);
+
+/* Stages of mla_decode, for timing them apart: a bit mask of the stages to enqueue.
+ * Running PLAN, then ATTEND, then COMBINE (in order, same arguments) equals mla_decode. */
+#define MLA_STAGE_PLAN 1
+#define MLA_STAGE_ATTEND 2
+#define MLA_STAGE_COMBINE 4
+MLA_API mla_status mla_decode_stages(const mla_config* cfg, int32_t stages, const void* q,
+                             const void* pool, const int32_t* block_table, int32_t max_blocks,
+                             int32_t num_blocks, const int32_t* seq_lens, int32_t batch,
+                             int32_t q_per_seq, void* workspace, size_t workspace_bytes,
+                             float* out_latent, float* lse, uint32_t* dev_err, void* stream);
+
+/*
+ * mla_output -- [B] Absorbing projections, [C] "rearrangement for calculating the final
+ * output": o[n, h, :] = W_UV[h] out_latent[n, h, :] (fp32 accumulation).
+ * out_latent (n_tokens, H, r) float32; w_uv (H, d_v, r) dtype (the nn.Linear(r, H*d_v)
+ * weight); o (n_tokens, H, d_v) dtype. W_O is not part of the library.
+ */
+MLA_API mla_status mla_output(const mla_config* cfg, const float* out_latent, const void* w_uv, void* o,
+                      int32_t n_tokens, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+MLA_API const char* mla_status_string(mla_status status);
+
+/* MLA_ABI_VERSION of the built library. */
+MLA_API int32_t mla_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

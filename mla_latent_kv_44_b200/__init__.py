@@ -1,0 +1,169 @@
+"""Python binding of libmla (MLA absorbed decode for B200, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA kernels of
+``libmla.so``. Tensors are passed as raw device pointers; PyTorch provides device memory and
+streams. Importing this module fails loudly when the library has not been built
+(``python -m mla_latent_kv_44_b200.build``); there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so")
+
+MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA, MLA_ERR_WORKSPACE = range(5)
+MLA_F32, MLA_BF16 = 0, 1
+DECODE_AUTO, DECODE_SIMT, DECODE_TENSOR = 0, 1, 2
+DEV_OOB_BLOCK, DEV_OOB_POS, DEV_WAIT_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
+STAGE_PLAN, STAGE_ATTEND, STAGE_COMBINE = 1, 2, 4
+STAGES_ALL = STAGE_PLAN | STAGE_ATTEND | STAGE_COMBINE
+
+_c_i32, _c_f32, _vp, _sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+
+class MlaConfig(ctypes.Structure):
+    _fields_ = [("num_heads", _c_i32), ("head_dim", _c_i32), ("head_dim_v", _c_i32),
+                ("kv_rank", _c_i32), ("rope_dim", _c_i32), ("block_size", _c_i32),
+                ("rope_base", _c_f32), ("rms_eps", _c_f32), ("softmax_scale", _c_f32),
+                ("dtype", _c_i32), ("decode_kernel", _c_i32)]
+
+
+class MlaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m mla_latent_kv_44_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(MlaConfig)
+    sig = {
+        "mla_absorb_query": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _c_i32, _vp]),
+        "mla_append_latent": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _vp,
+                                       _c_i32, _c_i32, _vp, _vp]),
+        "mla_decode_workspace_size": (_sz, [P, _c_i32, _c_i32]),
+        "mla_decode": (_c_i32, [P, _vp, _vp, _vp, _c_i32, _c_i32, _vp, _c_i32, _c_i32, _vp, _sz,
+                                _vp, _vp, _vp, _vp]),
+        "mla_decode_stages": (_c_i32, [P, _c_i32, _vp, _vp, _vp, _c_i32, _c_i32, _vp, _c_i32,
+                                       _c_i32, _vp, _sz, _vp, _vp, _vp, _vp]),
+        "mla_output": (_c_i32, [P, _vp, _vp, _vp, _c_i32, _vp]),
+        "mla_status_string": (ctypes.c_char_p, [_c_i32]),
+        "mla_abi_version": (_c_i32, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+@dataclass
+class Config:
+    """Shape and numerics of one MLA layer's decode (mirrors ``mla_config``)."""
+
+    num_heads: int
+    head_dim: int
+    kv_rank: int
+    rope_dim: int
+    block_size: int
+    dtype: str = "bf16"            # "bf16" or "f32"
+    head_dim_v: int = 0            # 0: same as head_dim
+    rope_base: float = 10000.0
+    rms_eps: float = 1e-6
+    softmax_scale: float = 0.0     # 0: 1 / sqrt(head_dim + rope_dim)
+    decode_kernel: int = DECODE_AUTO
+
+    def c(self) -> MlaConfig:
+        scale = self.softmax_scale or 1.0 / math.sqrt(self.head_dim + self.rope_dim)
+        return MlaConfig(self.num_heads, self.head_dim, self.head_dim_v or self.head_dim,
+                         self.kv_rank, self.rope_dim, self.block_size, self.rope_base,
+                         self.rms_eps, scale, MLA_BF16 if self.dtype == "bf16" else MLA_F32,
+                         self.decode_kernel)
+
+    @property
+    def row_width(self) -> int:
+        return self.kv_rank + self.rope_dim
+
+    @property
+    def torch_dtype(self):
+        import torch
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+
+def status_string(status: int) -> str:
+    return lib.mla_status_string(status).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _check(st: int, where: str):
+    if st != MLA_OK:
+        raise MlaError(st, where)
+
+
+def absorb_query(cfg: Config, q_nope, q_rope, pos, w_uk, q_out, stream=None):
+    """mla_absorb_query: q_out[n, h] = [W_UK[h]^T q_nope[n, h] || RoPE(q_rope[n, h], pos[n])]."""
+    c = cfg.c()
+    _check(lib.mla_absorb_query(ctypes.byref(c), _ptr(q_nope), _ptr(q_rope), _ptr(pos),
+                                _ptr(w_uk), _ptr(q_out), int(q_nope.shape[0]), _stream(stream)),
+           "mla_absorb_query")
+
+
+def append_latent(cfg: Config, ckv_raw, krope_raw, gamma, seq_idx, pos, block_table, pool,
+                  dev_err, stream=None):
+    """mla_append_latent: write [RMSNorm(c_kv) * gamma || RoPE(k_rope)] rows into the pool."""
+    c = cfg.c()
+    _check(lib.mla_append_latent(ctypes.byref(c), _ptr(ckv_raw), _ptr(krope_raw), _ptr(gamma),
+                                 _ptr(seq_idx), _ptr(pos), _ptr(block_table),
+                                 int(block_table.shape[0]), int(block_table.shape[1]), _ptr(pool),
+                                 int(pool.shape[0]), int(ckv_raw.shape[0]), _ptr(dev_err),
+                                 _stream(stream)), "mla_append_latent")
+
+
+def decode_workspace_size(cfg: Config, batch: int, q_per_seq: int) -> int:
+    c = cfg.c()
+    return int(lib.mla_decode_workspace_size(ctypes.byref(c), batch, q_per_seq))
+
+
+def decode(cfg: Config, q, pool, block_table, seq_lens, q_per_seq: int, workspace, out_latent,
+           lse, dev_err, stream=None, stages: int = STAGES_ALL):
+    """mla_decode (or a subset of its stages): split-KV absorbed attention over the pool."""
+    c = cfg.c()
+    _check(lib.mla_decode_stages(ctypes.byref(c), stages, _ptr(q), _ptr(pool), _ptr(block_table),
+                                 int(block_table.shape[1]), int(pool.shape[0]), _ptr(seq_lens),
+                                 int(seq_lens.shape[0]), q_per_seq, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _ptr(out_latent),
+                                 _ptr(lse), _ptr(dev_err), _stream(stream)), "mla_decode")
+
+
+def output(cfg: Config, out_latent, w_uv, o, stream=None):
+    """mla_output: o[n, h] = W_UV[h] out_latent[n, h]."""
+    c = cfg.c()
+    _check(lib.mla_output(ctypes.byref(c), _ptr(out_latent), _ptr(w_uv), _ptr(o),
+                          int(out_latent.shape[0]), _stream(stream)), "mla_output")
+
+
+def abi_version() -> int:
+    return int(lib.mla_abi_version())

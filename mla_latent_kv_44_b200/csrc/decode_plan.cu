@@ -1,0 +1,188 @@
+// Split-KV schedule and log-sum-exp combine of mla_decode.
+//
+// Every (sequence b, query token t) row group attends L = seq_lens[b] - T + 1 + t rows; its
+// rows are cut into 64-row chunks and all chunks of the call are laid end to end. The planner
+// cuts that list into R = min(74, chunks) ranges of equal size (range q starts at chunk
+// floor(q * C / R)). A row group touched by one range is a single segment whose result goes
+// straight to the output; a row group crossed by range boundaries becomes several segments
+// whose softmax-normalised partial results (with their log-sum-exp) are merged by the combine
+// kernel. Integer work only: the schedule is a pure function of seq_lens.
+#include "common.cuh"
+
+namespace mla {
+
+// Number of range starts strictly below chunk x: #{q in [0,R) : floor(q*C/R) < x}.
+__device__ __forceinline__ int starts_below(int64_t x, int64_t R, int64_t C) {
+  if (x <= 0 || C <= 0) return 0;
+  const int64_t v = (x * R + C - 1) / C;
+  return (int)(v < R ? v : R);
+}
+
+__device__ __forceinline__ int range_start(int64_t q, int64_t R, int64_t C) {
+  return (int)((q * C) / R);
+}
+
+constexpr int kPlanThreads = 1024;
+
+// Inclusive block scan of two ints over kPlanThreads threads.
+__device__ void block_scan2(int* s_a, int* s_b, int& a, int& b) {
+  const int tid = threadIdx.x;
+  s_a[tid] = a;
+  s_b[tid] = b;
+  __syncthreads();
+  for (int off = 1; off < kPlanThreads; off <<= 1) {
+    const int va = tid >= off ? s_a[tid - off] : 0;
+    const int vb = tid >= off ? s_b[tid - off] : 0;
+    __syncthreads();
+    s_a[tid] += va;
+    s_b[tid] += vb;
+    __syncthreads();
+  }
+  a = s_a[tid];
+  b = s_b[tid];
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p) {
+  __shared__ int s_a[kPlanThreads], s_b[kPlanThreads];
+  __shared__ int s_carry_a, s_carry_b;
+  const int tid = threadIdx.x;
+  const int64_t cap = (int64_t)p.max_blocks * p.bs;
+
+  // Pass 1: attended lengths, chunk counts, exclusive prefix of chunk counts.
+  if (tid == 0) s_carry_a = 0;
+  __syncthreads();
+  for (int base = 0; base < p.BT; base += kPlanThreads) {
+    const int bt = base + tid;
+    int nch = 0;
+    if (bt < p.BT) {
+      const int b = bt / p.T, t = bt - b * p.T;
+      const int sl = p.seq_lens[b];
+      int len = 0;
+      if (sl < p.T || (int64_t)sl > cap) {
+        if (t == 0) set_error(p.err, MLA_DEV_BAD_LENGTH);
+      } else {
+        len = sl - p.T + 1 + t;
+      }
+      nch = (len + kChunk - 1) / kChunk;
+      p.bt_len[bt] = len;
+    }
+    int inc = nch, dummy = 0;
+    block_scan2(s_a, s_b, inc, dummy);
+    if (bt < p.BT) p.bt_chunk0[bt] = s_carry_a + inc - nch;
+    __syncthreads();
+    if (tid == kPlanThreads - 1) s_carry_a += inc;
+    __syncthreads();
+  }
+  const int C = s_carry_a;
+  const int R = C < kRanges ? C : kRanges;
+  __syncthreads();
+
+  // Pass 2: segments per row group, their global indices and partial-result slots.
+  if (tid == 0) { s_carry_a = 0; s_carry_b = 0; }
+  __syncthreads();
+  for (int base = 0; base < p.BT; base += kPlanThreads) {
+    const int bt = base + tid;
+    int nseg = 0, nslot = 0, x = 0, e = 0;
+    if (bt < p.BT) {
+      const int len = p.bt_len[bt];
+      const int nch = (len + kChunk - 1) / kChunk;
+      x = p.bt_chunk0[bt];
+      e = x + nch;
+      if (nch > 0) nseg = 1 + starts_below(e, R, C) - starts_below(x + 1, R, C);
+      nslot = nseg >= 2 ? nseg : 0;
+    }
+    int inc_seg = nseg, inc_slot = nslot;
+    block_scan2(s_a, s_b, inc_seg, inc_slot);
+    if (bt < p.BT) {
+      const int first = s_carry_a + inc_seg - nseg;
+      const int slot0 = s_carry_b + inc_slot - nslot;
+      p.bt_first[bt] = first;
+      p.bt_nseg[bt] = nseg;
+      // cut points of this row group: x, the range starts strictly inside (x, e), e
+      int q = starts_below(x + 1, R, C);  // first range starting after x
+      int lo = x;
+      for (int k = 0; k < nseg; ++k) {
+        const int hi = (k == nseg - 1) ? e : range_start(q, R, C);
+        Segment sg;
+        sg.bt = bt;
+        sg.chunk_lo = lo;
+        sg.chunk_hi = hi;
+        sg.slot = nseg >= 2 ? slot0 + k : -1;
+        p.segments[first + k] = sg;
+        // a range starting exactly here begins with this segment
+        const int qs = starts_below(lo + 1, R, C) - 1;  // range containing chunk lo
+        if (qs >= 0 && range_start(qs, R, C) == lo) p.range_begin[qs] = first + k;
+        lo = hi;
+        ++q;
+      }
+    }
+    __syncthreads();
+    if (tid == kPlanThreads - 1) { s_carry_a += inc_seg; s_carry_b += inc_slot; }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    p.header[0] = s_carry_a;  // segments
+    p.header[1] = R;          // ranges in use
+    p.header[2] = C;          // chunks
+    p.range_begin[R] = s_carry_a;
+  }
+}
+
+cudaError_t launch_plan(const DecodeParams& p, cudaStream_t st) {
+  plan_kernel<<<1, kPlanThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
+// Combine: out = sum_i exp(lse_i - L) * o_i, L = log sum_i exp(lse_i), in segment order.
+// One CTA per (row group, 4 heads); row groups with a single segment were written directly by
+// the attention kernel and are skipped; row groups with an invalid length get 0 and -inf.
+// ------------------------------------------------------------------------------------------
+constexpr int kCombineHeads = 4;
+
+__global__ void __launch_bounds__(128) combine_kernel(DecodeParams p) {
+  const int bt = blockIdx.x;
+  const int nseg = p.bt_nseg[bt];
+  if (nseg == 1) return;
+  const int first = p.bt_first[bt];
+  for (int hh = 0; hh < kCombineHeads; ++hh) {
+    const int h = blockIdx.y * kCombineHeads + hh;
+    if (h >= p.H) break;
+    float* dst = p.out + ((size_t)bt * p.H + h) * p.r;
+    if (nseg == 0) {
+      for (int d = threadIdx.x; d < p.r; d += blockDim.x) dst[d] = 0.f;
+      if (threadIdx.x == 0 && p.lse) p.lse[(size_t)bt * p.H + h] = -INFINITY;
+      continue;
+    }
+    float mx = -INFINITY;
+    for (int k = 0; k < nseg; ++k)
+      mx = fmaxf(mx, p.part_lse[(size_t)p.segments[first + k].slot * p.H + h]);
+    if (mx == -INFINITY) {  // every part empty (all its blocks were rejected): no rows
+      for (int d = threadIdx.x; d < p.r; d += blockDim.x) dst[d] = 0.f;
+      if (threadIdx.x == 0 && p.lse) p.lse[(size_t)bt * p.H + h] = -INFINITY;
+      continue;
+    }
+    float z = 0.f;
+    for (int k = 0; k < nseg; ++k)
+      z += expf(p.part_lse[(size_t)p.segments[first + k].slot * p.H + h] - mx);
+    const float L = mx + logf(z);
+    for (int d = threadIdx.x; d < p.r; d += blockDim.x) {
+      float acc = 0.f;
+      for (int k = 0; k < nseg; ++k) {
+        const int slot = p.segments[first + k].slot;
+        const float w = expf(p.part_lse[(size_t)slot * p.H + h] - L);
+        acc = fmaf(w, p.part_o[((size_t)slot * p.H + h) * p.r + d], acc);
+      }
+      dst[d] = acc;
+    }
+    if (threadIdx.x == 0 && p.lse) p.lse[(size_t)bt * p.H + h] = L;
+  }
+}
+
+cudaError_t launch_combine(const DecodeParams& p, cudaStream_t st) {
+  dim3 grid(p.BT, (p.H + kCombineHeads - 1) / kCombineHeads);
+  combine_kernel<<<grid, 128, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -1,0 +1,173 @@
+// C ABI of libmla: argument validation, workspace carving and kernel dispatch.
+// Every entry point validates synchronously before any CUDA call and only enqueues work.
+#include <cmath>
+#include <cstdint>
+
+#include "common.cuh"
+
+using namespace mla;
+
+namespace {
+
+bool valid_config(const mla_config* c) {
+  if (!c) return false;
+  if (c->num_heads < 1 || c->num_heads > 4096) return false;
+  if (c->head_dim < 1 || c->head_dim > 1024) return false;
+  if (c->head_dim_v < 1 || c->head_dim_v > 1024) return false;
+  if (c->kv_rank < 32 || c->kv_rank > 1024 || c->kv_rank % 32 != 0) return false;
+  if (c->rope_dim < 0 || c->rope_dim > 256 || c->rope_dim % 2 != 0) return false;
+  if ((c->kv_rank + c->rope_dim) % 8 != 0) return false;
+  if (c->block_size < 1) return false;
+  if (c->dtype != MLA_F32 && c->dtype != MLA_BF16) return false;
+  if (c->decode_kernel < MLA_DECODE_AUTO || c->decode_kernel > MLA_DECODE_TENSOR) return false;
+  if (!std::isfinite(c->softmax_scale) || !(c->softmax_scale > 0.f)) return false;
+  if (!std::isfinite(c->rope_base) || !(c->rope_base > 0.f)) return false;
+  if (!std::isfinite(c->rms_eps) || c->rms_eps < 0.f) return false;
+  return true;
+}
+
+mla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
+
+mla_status mla_absorb_query(const mla_config* cfg, const void* q_nope, const void* q_rope,
+                            const int32_t* pos, const void* w_uk, void* q_out, int32_t n_tokens,
+                            void* stream) {
+  if (!valid_config(cfg) || n_tokens < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MLA_OK;
+  if (!q_nope || !w_uk || !q_out || !pos || (cfg->rope_dim > 0 && !q_rope))
+    return MLA_ERR_INVALID_ARG;
+  if (n_tokens > (1 << 24)) return MLA_ERR_UNSUPPORTED;
+  return from_cuda(launch_absorb(*cfg, q_nope, q_rope, pos, w_uk, q_out, n_tokens,
+                                 (cudaStream_t)stream));
+}
+
+mla_status mla_append_latent(const mla_config* cfg, const void* ckv_raw, const void* krope_raw,
+                             const float* gamma, const int32_t* seq_idx, const int32_t* pos,
+                             const int32_t* block_table, int32_t batch, int32_t max_blocks,
+                             void* pool, int32_t num_blocks, int32_t n_tokens, uint32_t* dev_err,
+                             void* stream) {
+  if (!valid_config(cfg) || n_tokens < 0 || batch < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MLA_OK;
+  if (!ckv_raw || (cfg->rope_dim > 0 && !krope_raw) || !gamma || !seq_idx || !pos ||
+      !block_table || !pool || !dev_err)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || max_blocks < 1 || num_blocks < 1) return MLA_ERR_INVALID_ARG;
+  if (n_tokens > (1 << 26)) return MLA_ERR_UNSUPPORTED;
+  return from_cuda(launch_append(*cfg, ckv_raw, krope_raw, gamma, seq_idx, pos, block_table,
+                                 batch, max_blocks, pool, num_blocks, n_tokens, dev_err,
+                                 (cudaStream_t)stream));
+}
+
+size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t q_per_seq) {
+  if (!valid_config(cfg) || batch < 1 || q_per_seq < 1) return 0;
+  const int64_t bt = (int64_t)batch * q_per_seq;
+  if (bt > (1 << 24)) return 0;
+  return workspace_layout(cfg->num_heads, cfg->kv_rank, (int)bt).total;
+}
+
+mla_status mla_decode_stages(const mla_config* cfg, int32_t stages, const void* q,
+                             const void* pool, const int32_t* block_table, int32_t max_blocks,
+                             int32_t num_blocks, const int32_t* seq_lens, int32_t batch,
+                             int32_t q_per_seq, void* workspace, size_t workspace_bytes,
+                             float* out_latent, float* lse, uint32_t* dev_err, void* stream) {
+  if (!valid_config(cfg) || batch < 0 || q_per_seq < 1) return MLA_ERR_INVALID_ARG;
+  if (stages & ~(MLA_STAGE_PLAN | MLA_STAGE_ATTEND | MLA_STAGE_COMBINE)) return MLA_ERR_INVALID_ARG;
+  if (batch == 0 || stages == 0) return MLA_OK;
+  if (!q || !pool || !block_table || !seq_lens || !workspace || !out_latent || !dev_err)
+    return MLA_ERR_INVALID_ARG;
+  if (max_blocks < 1 || num_blocks < 1) return MLA_ERR_INVALID_ARG;
+  const int64_t bt = (int64_t)batch * q_per_seq;
+  if (bt > (1 << 24)) return MLA_ERR_UNSUPPORTED;
+  const size_t need = mla_decode_workspace_size(cfg, batch, q_per_seq);
+  if (need == 0) return MLA_ERR_INVALID_ARG;
+  if (workspace_bytes < need || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+  if (!aligned(pool, 16) || !aligned(q, 16)) return MLA_ERR_INVALID_ARG;
+
+  bool use_tc;
+  switch (cfg->decode_kernel) {
+    case MLA_DECODE_SIMT: use_tc = false; break;
+    case MLA_DECODE_TENSOR:
+      if (!tc_supported(*cfg)) return MLA_ERR_UNSUPPORTED;
+      use_tc = true;
+      break;
+    default: use_tc = tc_supported(*cfg); break;
+  }
+
+  const WorkspaceLayout L = workspace_layout(cfg->num_heads, cfg->kv_rank, (int)bt);
+  char* ws = static_cast<char*>(workspace);
+  DecodeParams p;
+  p.q = q;
+  p.pool = pool;
+  p.table = block_table;
+  p.seq_lens = seq_lens;
+  p.out = out_latent;
+  p.lse = lse;
+  p.err = dev_err;
+  p.header = reinterpret_cast<int32_t*>(ws + L.header);
+  p.range_begin = reinterpret_cast<int32_t*>(ws + L.range_begin);
+  p.segments = reinterpret_cast<Segment*>(ws + L.segments);
+  p.bt_first = reinterpret_cast<int32_t*>(ws + L.bt_first);
+  p.bt_nseg = reinterpret_cast<int32_t*>(ws + L.bt_nseg);
+  p.bt_len = reinterpret_cast<int32_t*>(ws + L.bt_len);
+  p.bt_chunk0 = reinterpret_cast<int32_t*>(ws + L.bt_chunk0);
+  p.part_lse = reinterpret_cast<float*>(ws + L.part_lse);
+  p.part_o = reinterpret_cast<float*>(ws + L.part_o);
+  p.H = cfg->num_heads;
+  p.r = cfg->kv_rank;
+  p.dr = cfg->rope_dim;
+  p.D = cfg->kv_rank + cfg->rope_dim;
+  p.bs = cfg->block_size;
+  p.max_blocks = max_blocks;
+  p.num_blocks = num_blocks;
+  p.batch = batch;
+  p.T = q_per_seq;
+  p.BT = (int)bt;
+  p.scale = cfg->softmax_scale;
+
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (stages & MLA_STAGE_PLAN) e = launch_plan(p, st);
+  if (e == cudaSuccess && (stages & MLA_STAGE_ATTEND))
+    e = use_tc ? launch_attend_tc(*cfg, p, st) : launch_attend_simt(*cfg, p, st);
+  if (e == cudaSuccess && (stages & MLA_STAGE_COMBINE)) e = launch_combine(p, st);
+  return from_cuda(e);
+}
+
+mla_status mla_decode(const mla_config* cfg, const void* q, const void* pool,
+                      const int32_t* block_table, int32_t max_blocks, int32_t num_blocks,
+                      const int32_t* seq_lens, int32_t batch, int32_t q_per_seq, void* workspace,
+                      size_t workspace_bytes, float* out_latent, float* lse, uint32_t* dev_err,
+                      void* stream) {
+  return mla_decode_stages(cfg, MLA_STAGE_PLAN | MLA_STAGE_ATTEND | MLA_STAGE_COMBINE, q, pool,
+                           block_table, max_blocks, num_blocks, seq_lens, batch, q_per_seq,
+                           workspace, workspace_bytes, out_latent, lse, dev_err, stream);
+}
+
+mla_status mla_output(const mla_config* cfg, const float* out_latent, const void* w_uv, void* o,
+                      int32_t n_tokens, void* stream) {
+  if (!valid_config(cfg) || n_tokens < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MLA_OK;
+  if (!out_latent || !w_uv || !o) return MLA_ERR_INVALID_ARG;
+  if (n_tokens > (1 << 24)) return MLA_ERR_UNSUPPORTED;
+  return from_cuda(launch_output(*cfg, out_latent, w_uv, o, n_tokens, (cudaStream_t)stream));
+}
+
+}  // extern "C"

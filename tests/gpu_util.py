@@ -1,0 +1,59 @@
+"""Helpers for the GPU parity tests: expected values come only from the CPU oracle."""
+import numpy as np
+import torch
+
+import mla_inputs as mi
+from oracle import compare, mla_ref as ref
+
+
+def oracle_sequence(state, b: int, form: str = "naive"):
+    """The oracle's result for sequence b of a DecodeState, from the same host inputs."""
+    w = state.w
+    ckv, kr, qn, qr = state.host_draws[b]
+    return ref.decode_sequence_from_raw(ckv, kr, qn, qr, state.w_uk_host, state.w_uv_host,
+                                        state.gamma_host, w.softmax_scale, w.rms_eps, w.rope_base,
+                                        store_bf16=(w.dtype == "bf16"), form=form)
+
+
+def check_sequence(state, b: int, form: str = "naive", lse_tol=None):
+    """Compare o, out_latent and lse of sequence b with the oracle; returns the error metrics."""
+    exp = oracle_sequence(state, b, form)
+    sl = state.tokens_of(b)
+    o = state.o[sl].float().cpu().numpy()
+    lat = state.out_latent[sl].cpu().numpy()
+    lse = state.lse[sl].cpu().numpy()
+    dt = state.w.dtype
+    ok_o, e_o = compare.within(o, exp.o, dt)
+    ok_l, e_l = compare.within(lat, exp.o_lat, dt)
+    e_lse = float(np.max(np.abs(lse - exp.lse)))
+    tol = lse_tol if lse_tol is not None else (2e-2 if dt == "bf16" else 1e-5 * max(1.0, float(np.max(np.abs(exp.lse)))))
+    assert ok_o, f"seq {b}: output error {e_o}"
+    assert ok_l, f"seq {b}: latent output error {e_l}"
+    assert e_lse <= tol, f"seq {b}: lse error {e_lse}"
+    return e_o, e_l, e_lse
+
+
+def dev_err(state) -> int:
+    torch.cuda.synchronize()
+    return int(state.dev_err.item())
+
+
+def layer_raw(w: mi.Workload, seed: int = 0):
+    """Projections of seeded hidden states by the oracle's front end (small workloads)."""
+    d = mi.layer_draw(w, seed)
+    p = ref.project_layer(d.x, w.num_heads, w.head_dim, w.rope_dim, d.w_dkv, d.w_kr, d.w_qr,
+                          w_q=d.w_q, w_dq=d.w_dq, w_uq=d.w_uq, gamma_q=d.gamma_q, eps=w.rms_eps)
+    rows = mi.total_rows(w, seed)
+    T = w.new_tokens
+    H = w.num_heads
+    raw = dict(w_uk=d.w_uk.reshape(H, w.head_dim, w.kv_rank).astype(np.float32),
+               w_uv=d.w_uv.reshape(H, w.head_dim_v, w.kv_rank).astype(np.float32),
+               gamma=d.gamma_kv.astype(np.float32), ckv_raw=[], krope_raw=[], q_nope=[],
+               q_rope_raw=[])
+    for b in range(w.batch):
+        n = int(rows[b])
+        raw["ckv_raw"].append(p.ckv_raw[b, :n].astype(np.float32))
+        raw["krope_raw"].append(p.krope_raw[b, :n].astype(np.float32))
+        raw["q_nope"].append(p.q_nope[b, n - T:n].astype(np.float32))
+        raw["q_rope_raw"].append(p.q_rope_raw[b, n - T:n].astype(np.float32))
+    return raw

@@ -1,0 +1,118 @@
+"""The C ABI library loads, exports every symbol the header declares, and validates arguments
+synchronously (no GPU needed: every call here fails validation before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+@pytest.fixture(scope="module")
+def mla():
+    from mla_latent_kv_44_b200 import build
+
+    build.build()
+    import mla_latent_kv_44_b200 as m
+
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("mla_absorb_query", "mla_append_latent", "mla_decode", "mla_output"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(mla):
+    lib = ctypes.CDLL(mla.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_abi_version_and_status_strings(mla):
+    assert mla.abi_version() == 1
+    assert mla.status_string(0) == "MLA_OK"
+    assert mla.status_string(4) == "MLA_ERR_WORKSPACE"
+    assert mla.status_string(99) == "MLA_ERR_UNKNOWN"
+
+
+def _cfg(mla, **kw):
+    base = dict(num_heads=128, head_dim=128, kv_rank=512, rope_dim=64, block_size=64)
+    base.update(kw)
+    return mla.Config(**base).c()
+
+
+def test_workspace_size_is_host_arithmetic(mla):
+    c = _cfg(mla)
+    n1 = mla.lib.mla_decode_workspace_size(ctypes.byref(c), 64, 1)
+    n4 = mla.lib.mla_decode_workspace_size(ctypes.byref(c), 64, 4)
+    assert n1 > 148 * 128 * 512 * 4           # partial outputs of 2 * 74 slots
+    assert n4 > n1 and n1 % 256 == 0
+    assert mla.lib.mla_decode_workspace_size(ctypes.byref(c), 0, 1) == 0
+    assert mla.lib.mla_decode_workspace_size(None, 64, 1) == 0
+
+
+@pytest.mark.parametrize("bad", [dict(kv_rank=48), dict(rope_dim=3), dict(num_heads=0),
+                                 dict(block_size=0), dict(dtype="f16")])
+def test_invalid_config_rejected(mla, bad):
+    kw = dict(num_heads=128, head_dim=128, kv_rank=512, rope_dim=64, block_size=64)
+    kw.update(bad)
+    cfg = mla.Config(**kw)
+    c = cfg.c()
+    if bad.get("dtype") == "f16":
+        c.dtype = 7
+    st = mla.lib.mla_absorb_query(ctypes.byref(c), 1, 1, 1, 1, 1, 4, None)
+    assert st == mla.MLA_ERR_INVALID_ARG
+
+
+def test_null_pointers_rejected_without_launch(mla):
+    c = _cfg(mla)
+    assert mla.lib.mla_absorb_query(ctypes.byref(c), None, 1, 1, 1, 1, 4, None) == 1
+    assert mla.lib.mla_output(ctypes.byref(c), None, 1, 1, 4, None) == 1
+    assert mla.lib.mla_append_latent(ctypes.byref(c), 1, 1, 1, 1, 1, 1, 2, 2, 1, 4, 8, None,
+                                     None) == 1
+    ws = mla.lib.mla_decode_workspace_size(ctypes.byref(c), 2, 1)
+    assert mla.lib.mla_decode(ctypes.byref(c), None, 256, 256, 2, 4, 256, 2, 1, 256, ws, 256,
+                              None, 256, None) == 1
+
+
+def test_workspace_too_small_or_misaligned(mla):
+    c = _cfg(mla)
+    ws = mla.lib.mla_decode_workspace_size(ctypes.byref(c), 2, 1)
+    args = (256, 256, 256, 2, 4, 256, 2, 1)
+    assert mla.lib.mla_decode(ctypes.byref(c), *args, 256, ws - 1, 256, None, 256, None) == 4
+    assert mla.lib.mla_decode(ctypes.byref(c), *args, 257, ws, 256, None, 256, None) == 4
+
+
+def test_empty_work_is_a_no_op(mla):
+    c = _cfg(mla)
+    assert mla.lib.mla_absorb_query(ctypes.byref(c), None, None, None, None, None, 0, None) == 0
+    assert mla.lib.mla_output(ctypes.byref(c), None, None, None, 0, None) == 0
+    assert mla.lib.mla_decode(ctypes.byref(c), None, None, None, 1, 1, None, 0, 1, None, 0, None,
+                              None, None, None) == 0
+
+
+def test_tensor_kernel_request_for_unsupported_shape(mla):
+    c = _cfg(mla, num_heads=16, kv_rank=64, rope_dim=32)
+    c.decode_kernel = mla.DECODE_TENSOR
+    ws = mla.lib.mla_decode_workspace_size(ctypes.byref(c), 2, 1)
+    st = mla.lib.mla_decode(ctypes.byref(c), 256, 256, 256, 2, 4, 256, 2, 1, 256, ws, 256, None,
+                            256, None)
+    assert st == mla.MLA_ERR_UNSUPPORTED
+
+
+def test_product_package_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "mla_latent_kv_44_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in re.findall(r"^\s*(?:from|import)\s+(\w+)", text, re.M), f
