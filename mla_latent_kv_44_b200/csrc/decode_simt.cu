@@ -23,8 +23,9 @@ attend_simt_kernel(DecodeParams p) {
   const Segment sg = p.segments[seg_id];
   const int bt = sg.bt, b = bt / p.T;
   const int len = p.bt_len[bt];
-  const int tok_lo = sg.chunk_lo * kChunk;
-  const int tok_hi = min(sg.chunk_hi * kChunk, len);
+  const int chunk0 = p.bt_chunk0[bt];  // segment chunks are numbered across all row groups
+  const int tok_lo = (sg.chunk_lo - chunk0) * kChunk;
+  const int tok_hi = min((sg.chunk_hi - chunk0) * kChunk, len);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y * kSimtHeads + warp;
   const bool active = h < p.H;

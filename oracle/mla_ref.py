@@ -374,3 +374,21 @@ def decode_sequence_from_raw(ckv_raw, krope_raw, q_nope, q_rope_raw, w_uk, w_uv,
     q_rope = rope_rotate(np.asarray(q_rope_raw, dtype=F64), qpos[:, None], base)
     fn = naive_decode if form == "naive" else absorbed_decode
     return fn(rows[:, :r], rows[:, r:], np.asarray(q_nope, dtype=F64), q_rope, w_uk, w_uv, scale)
+
+
+def decode_sequence_bf16_query(ckv_raw, krope_raw, q_nope, q_rope_raw, w_uk, w_uv, gamma,
+                               scale: float, eps: float, base: float) -> DecodeOut:
+    """Absorbed form with the packed query [q_lat || q_rope] stored in bfloat16.
+
+    On a bf16 model the absorbed query is a bfloat16 tensor like every other activation (the
+    module of "MLA from scratch in PyTorch" computes in its parameters' dtype); rounding it
+    once, to nearest even, separates that storage error -- which peaky attention amplifies --
+    from the error of the attention arithmetic itself. Everything else is float64.
+    """
+    L = np.asarray(ckv_raw).shape[0]
+    T = np.asarray(q_nope).shape[0]
+    r = np.asarray(ckv_raw).shape[1]
+    rows = cache_rows(ckv_raw, krope_raw, gamma, np.arange(L), eps, base, True)
+    Q = round_bf16(absorb_ref(q_nope, q_rope_raw, np.arange(L - T, L), w_uk, base))
+    lat = latent_attention(Q, rows, r, scale, T)
+    return DecodeOut(output_ref(lat.o_lat, w_uv), lat.o_lat, lat.lse)

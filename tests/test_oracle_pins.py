@@ -423,3 +423,47 @@ def test_needle_makes_attention_peaky():
     p = ref.softmax(s)
     assert p[0, :, j].max() > 0.5
     assert np.argmax(p[0].max(axis=1)) is not None
+
+
+# ----------------------------------------------------------------------------------------
+# The bf16-query form: only the query's storage differs from the absorbed form
+# ----------------------------------------------------------------------------------------
+
+def _emulate_bf16_path(Q, rows, r, scale, wuv):
+    """bf16 query, weights rounded to bf16 before the weighted sum, bf16 output."""
+    Qb = ref.round_bf16(Q)
+    s = np.einsum("thd,ld->thl", Qb, rows) * scale
+    pe = np.exp(s - s.max(-1, keepdims=True))
+    lat = np.einsum("thl,lj->thj", ref.round_bf16(pe), rows[:, :r]) / pe.sum(-1, keepdims=True)
+    return ref.round_bf16(ref.output_ref(lat, wuv)), lat
+
+
+@pytest.mark.parametrize("factor", [0.0, 4.0, 16.0])
+def test_bf16_query_form(factor):
+    w = mi.scaled(mi.WORKLOADS["small_bf16"], batch=1, cached=400)
+    rows_n = int(mi.total_rows(w)[0])
+    d = mi.sequence_draw(w, 0, rows_n)
+    if factor:
+        mi.plant_needle(w, d, factor=factor)
+    wuk, wuv = (mi.storage_round(w, x) for x in mi.up_projection_weights(w))
+    ckv, kr, qn, qr = (mi.storage_round(w, x) for x in (d.ckv_raw, d.krope_raw, d.q_nope,
+                                                         d.q_rope_raw))
+    g = np.ones(w.kv_rank)
+    args = (ckv, kr, qn, qr, wuk, wuv, g, w.softmax_scale, w.rms_eps, w.rope_base)
+    exact = ref.decode_sequence_from_raw(*args, True, "absorbed")
+    qb = ref.decode_sequence_bf16_query(*args)
+    # identical to the absorbed form when the query is already bf16-representable
+    Q = ref.absorb_ref(qn, qr, np.array([rows_n - 1]), wuk, w.rope_base)
+    rows = ref.cache_rows(ckv, kr, g, np.arange(rows_n), w.rms_eps, w.rope_base, True)
+    direct = ref.latent_attention(ref.round_bf16(Q), rows, w.kv_rank, w.softmax_scale, 1)
+    assert np.max(np.abs(direct.o_lat - qb.o_lat)) < 1e-12
+    # an emulation of the bf16 path's own roundings stays within 2e-2 of the bf16-query form
+    o, lat = _emulate_bf16_path(Q, rows, w.kv_rank, w.softmax_scale, wuv)
+    assert compare.within(o, qb.o, "bf16")[0] and compare.within(lat, qb.o_lat, "bf16")[0]
+    # and a head swap does not
+    sw = o.copy()
+    sw[:, [0, 1]] = sw[:, [1, 0]]
+    assert not compare.within(sw, qb.o, "bf16")[0]
+    # the query's storage is the whole difference from the exact form (small when diffuse)
+    if not factor:
+        assert compare.within(qb.o, exact.o, "bf16")[0]
