@@ -2,8 +2,9 @@
 
 Argument marshalling only: every step of the computation runs in the CUDA kernels of
 ``libmla.so``. Tensors are passed as raw device pointers; PyTorch provides device memory and
-streams. Importing this module fails loudly when the library has not been built
-(``python -m mla_latent_kv_44_b200.build``); there is no fallback.
+streams. The library is loaded on the first call (so that the build step can import this
+package before the library exists); that call fails loudly when the library has not been
+built (``python -m mla_latent_kv_44_b200.build``). There is no fallback.
 """
 from __future__ import annotations
 
@@ -63,7 +64,18 @@ def _load():
     return lib
 
 
-lib = _load()
+class _Lib:
+    """libmla.so, loaded on first use."""
+
+    _handle = None
+
+    def __getattr__(self, name):
+        if _Lib._handle is None:
+            _Lib._handle = _load()
+        return getattr(_Lib._handle, name)
+
+
+lib = _Lib()
 
 
 @dataclass

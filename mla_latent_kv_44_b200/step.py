@@ -37,7 +37,7 @@ class DecodeState:
 
     def __init__(self, w: mi.Workload, seed: int = 0, device: str = "cuda",
                  decode_kernel: int = DECODE_AUTO, raw: Optional[dict] = None,
-                 needle: bool = False, gamma_perturbed: bool = False, spare_blocks: int = 0,
+                 needle: float = 0.0, gamma_perturbed: bool = False, spare_blocks: int = 0,
                  sequences: Optional[Sequence[int]] = None):
         self.w = w
         self.device = torch.device(device)
@@ -80,7 +80,7 @@ class DecodeState:
             if raw is None:
                 d = mi.sequence_draw(w, b, n, seed)
                 if needle:
-                    self.needle_rows[b] = mi.plant_needle(w, d, seed)
+                    self.needle_rows[b] = mi.plant_needle(w, d, seed, factor=needle)
                 ckv, kr, q1, q2 = d.ckv_raw, d.krope_raw, d.q_nope, d.q_rope_raw
             else:
                 ckv, kr = raw["ckv_raw"][b][:n], raw["krope_raw"][b][:n]

@@ -19,10 +19,9 @@ def check_sequence(state, b: int, form: str = "naive", lse_tol=None, peaky: bool
     """Compare o, out_latent and lse of sequence b with the oracle; returns the error metrics.
 
     Tolerance: fp32 1e-5 relative; bf16 2e-2 on unit-scaled outputs (oracle.compare.within).
-    peaky: the inputs concentrate attention, which amplifies the bf16 storage of the absorbed
-    query; the kernel's result must then match the oracle's absorbed form with that query
-    rounded to bf16 within 2e-2, and its distance from the naive form may exceed the naive
-    form's distance from that bf16-query form by at most 2e-2.
+    peaky: one planted row takes most of the attention weight, which amplifies one-ulp
+    rounding differences of the bf16 query; the elementwise tolerance of
+    oracle.compare.peaky_tolerance applies instead.
     """
     exp = oracle_sequence(state, b, form)
     sl = state.tokens_of(b)
@@ -32,18 +31,19 @@ def check_sequence(state, b: int, form: str = "naive", lse_tol=None, peaky: bool
     dt = state.w.dtype
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lat)), f"seq {b}: non-finite output"
     if peaky:
+        # one needle row dominates: allow the first-order effect of a one-ulp rounding
+        # difference in the query or in that row on its score (oracle.compare.peaky_tolerance)
         w = state.w
         ckv, kr, qn, qr = state.host_draws[b]
-        qb = ref.decode_sequence_bf16_query(ckv, kr, qn, qr, state.w_uk_host, state.w_uv_host,
-                                            state.gamma_host, w.softmax_scale, w.rms_eps,
-                                            w.rope_base)
-        for got, want, naive in ((o, qb.o, exp.o), (lat, qb.o_lat, exp.o_lat)):
-            ok, e = compare.within(got, want, dt)
-            assert ok, f"seq {b}: error {e} against the bf16-query oracle"
-            e_gpu = compare.per_vector_scaled_error(got, naive)
-            e_q = compare.per_vector_scaled_error(want, naive)
-            assert e_gpu <= e_q + compare.BF16_SCALED_TOL, (
-                f"seq {b}: {e_gpu} from the naive form, bf16 query alone explains {e_q}")
+        n = ckv.shape[0]
+        rows = ref.cache_rows(ckv, kr, state.gamma_host, np.arange(n), w.rms_eps, w.rope_base,
+                              True)
+        Q = ref.absorb_ref(qn, qr, np.arange(n - w.new_tokens, n), state.w_uk_host, w.rope_base)
+        tol_o, tol_l = compare.peaky_tolerance(Q, rows, state.w_uv_host, w.kv_rank,
+                                               w.softmax_scale, state.needle_rows[b], exp.o,
+                                               exp.o_lat)
+        assert np.all(np.abs(o - exp.o) <= tol_o), f"seq {b}: output outside the needle tolerance"
+        assert np.all(np.abs(lat - exp.o_lat) <= tol_l), f"seq {b}: latent outside the needle tolerance"
         e_o = e_l = 0.0
     else:
         ok_o, e_o = compare.within(o, exp.o, dt)

@@ -65,7 +65,7 @@ def test_needle_peaky_attention(mla, name):
     w = mi.WORKLOADS[name]
     if name == "dsv2":
         w = mi.scaled(w, batch=2, cached=1000)
-    st = DecodeState(w, needle=True, gamma_perturbed=True)
+    st = DecodeState(w, needle=8.0, gamma_perturbed=True)
     st.step()
     assert dev_err(st) == 0
     for b in range(w.batch):

@@ -413,7 +413,7 @@ def test_needle_makes_attention_peaky():
     w = mi.scaled(mi.WORKLOADS["small_bf16"], batch=1, cached=300)
     rows = int(mi.total_rows(w)[0])
     d = mi.sequence_draw(w, 0, rows)
-    j = mi.plant_needle(w, d)
+    j = mi.plant_needle(w, d, factor=8.0)
     wuk, wuv = mi.up_projection_weights(w)
     c = ref.cache_rows(d.ckv_raw, d.krope_raw, np.ones(w.kv_rank), np.arange(rows), w.rms_eps,
                        w.rope_base, True)
@@ -467,3 +467,35 @@ def test_bf16_query_form(factor):
     # the query's storage is the whole difference from the exact form (small when diffuse)
     if not factor:
         assert compare.within(qb.o, exact.o, "bf16")[0]
+
+
+@pytest.mark.parametrize("factor", [4.0, 8.0, 16.0])
+def test_peaky_tolerance_admits_one_ulp_query_differences_only(factor):
+    w = mi.scaled(mi.WORKLOADS["small_bf16"], batch=1, cached=400)
+    n = int(mi.total_rows(w)[0])
+    d = mi.sequence_draw(w, 0, n)
+    j = mi.plant_needle(w, d, factor=factor)
+    wuk, wuv = (mi.storage_round(w, x) for x in mi.up_projection_weights(w))
+    ckv, kr, qn, qr = (mi.storage_round(w, x) for x in (d.ckv_raw, d.krope_raw, d.q_nope,
+                                                         d.q_rope_raw))
+    g = np.ones(w.kv_rank)
+    exact = ref.decode_sequence_from_raw(ckv, kr, qn, qr, wuk, wuv, g, w.softmax_scale,
+                                         w.rms_eps, w.rope_base, True)
+    rows = ref.cache_rows(ckv, kr, g, np.arange(n), w.rms_eps, w.rope_base, True)
+    Q = ref.absorb_ref(qn, qr, np.array([n - 1]), wuk, w.rope_base)
+    tol_o, tol_l = compare.peaky_tolerance(Q, rows, wuv, w.kv_rank, w.softmax_scale, j,
+                                           exact.o, exact.o_lat)
+    # a bf16 query rounded one ulp the other way in a random tenth of its elements
+    rng = np.random.default_rng(5)
+    Qb = ref.round_bf16(Q)
+    flip = rng.random(Q.shape) < 0.1
+    Qb = np.where(flip, Qb + np.sign(Q - Qb + 1e-300) * compare.bf16_ulp(Qb), Qb)
+    lat = ref.latent_attention(Qb, rows, w.kv_rank, w.softmax_scale, 1)
+    o = ref.output_ref(lat.o_lat, wuv)
+    assert np.all(np.abs(o - exact.o) <= tol_o)
+    assert np.all(np.abs(lat.o_lat - exact.o_lat) <= tol_l)
+    # but not a head swap, nor a zero output
+    sw = exact.o.copy()
+    sw[:, [0, 1]] = sw[:, [1, 0]]
+    assert not np.all(np.abs(sw - exact.o) <= tol_o)
+    assert not np.all(np.abs(exact.o) <= tol_o)
