@@ -154,6 +154,35 @@ MLA_API mla_status mla_decode_stages(const mla_config* cfg, int32_t stages, cons
                              float* out_latent, float* lse, uint32_t* dev_err, void* stream);
 
 /*
+ * Size of the device array that mla_decode_static_workspace uses as its workspace: 40 MiB,
+ * enough for the DeepSeek-V2 shape (H = 128, r = 512) at any batch up to several thousand
+ * (query token, sequence) pairs.
+ */
+#define MLA_STATIC_WORKSPACE_BYTES (40u << 20)
+
+/*
+ * mla_decode_static_workspace -- no counterpart on the pages: a library-side addition.
+ * Exactly mla_decode (same arguments, same kernels, same results) without the workspace
+ * arguments, for callers that cannot allocate device memory themselves: a host program with
+ * no device allocator of its own, or a decode loop that must not call cudaMalloc because it
+ * synchronises the device. The workspace is a file-scope device array of
+ * MLA_STATIC_WORKSPACE_BYTES that every GPU loading the library holds until exit. This call
+ * allocates nothing (no cudaMalloc, no cudaFree, no allocating library routine).
+ *   - Returns MLA_ERR_WORKSPACE when mla_decode_workspace_size(cfg, batch, q_per_seq) exceeds
+ *     MLA_STATIC_WORKSPACE_BYTES; nothing is launched.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     with that device current; make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents: calls that overlap
+ *     on the GPU (other streams, other threads) race and must be serialised by the caller.
+ */
+MLA_API mla_status mla_decode_static_workspace(const mla_config* cfg, const void* q,
+                                               const void* pool, const int32_t* block_table,
+                                               int32_t max_blocks, int32_t num_blocks,
+                                               const int32_t* seq_lens, int32_t batch,
+                                               int32_t q_per_seq, float* out_latent, float* lse,
+                                               uint32_t* dev_err, void* stream);
+
+/*
  * mla_output -- [B] Absorbing projections, [C] "rearrangement for calculating the final
  * output": o[n, h, :] = W_UV[h] out_latent[n, h, :] (fp32 accumulation).
  * out_latent (n_tokens, H, r) float32; w_uv (H, d_v, r) dtype (the nn.Linear(r, H*d_v)

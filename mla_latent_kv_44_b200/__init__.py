@@ -16,6 +16,7 @@ from dataclasses import dataclass
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so")
 
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA, MLA_ERR_WORKSPACE = range(5)
+STATIC_WORKSPACE_BYTES = 40 << 20
 MLA_F32, MLA_BF16 = 0, 1
 DECODE_AUTO, DECODE_SIMT, DECODE_TENSOR = 0, 1, 2
 DEV_OOB_BLOCK, DEV_OOB_POS, DEV_WAIT_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
@@ -54,6 +55,8 @@ def _load():
         "mla_decode_stages": (_c_i32, [P, _c_i32, _vp, _vp, _vp, _c_i32, _c_i32, _vp, _c_i32,
                                        _c_i32, _vp, _sz, _vp, _vp, _vp, _vp]),
         "mla_output": (_c_i32, [P, _vp, _vp, _vp, _c_i32, _vp]),
+        "mla_decode_static_workspace": (_c_i32, [P, _vp, _vp, _vp, _c_i32, _c_i32, _vp, _c_i32,
+                                                 _c_i32, _vp, _vp, _vp, _vp]),
         "mla_status_string": (ctypes.c_char_p, [_c_i32]),
         "mla_abi_version": (_c_i32, []),
     }
@@ -168,6 +171,19 @@ def decode(cfg: Config, q, pool, block_table, seq_lens, q_per_seq: int, workspac
                                  int(seq_lens.shape[0]), q_per_seq, _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _ptr(out_latent),
                                  _ptr(lse), _ptr(dev_err), _stream(stream)), "mla_decode")
+
+
+def decode_static_workspace(cfg: Config, q, pool, block_table, seq_lens, q_per_seq: int,
+                            out_latent, lse, dev_err, stream=None):
+    """mla_decode_static_workspace: mla_decode with the library's own fixed device workspace,
+    for callers that cannot allocate device memory (see include/mla.h)."""
+    c = cfg.c()
+    _check(lib.mla_decode_static_workspace(ctypes.byref(c), _ptr(q), _ptr(pool),
+                                           _ptr(block_table), int(block_table.shape[1]),
+                                           int(pool.shape[0]), _ptr(seq_lens),
+                                           int(seq_lens.shape[0]), q_per_seq, _ptr(out_latent),
+                                           _ptr(lse), _ptr(dev_err), _stream(stream)),
+           "mla_decode_static_workspace")
 
 
 def output(cfg: Config, out_latent, w_uv, o, stream=None):
