@@ -13,7 +13,8 @@
 // CTAs therefore shares every work range. CTA c loads only its half of each row -- latent dims
 // [256c, 256c + 256) and RoPE dims [32c, 32c + 32) -- so the pair reads each cache byte once:
 //   * both CTAs compute a partial S over their 288 dims (Q half resident in TMEM as the A
-//     operand), swap the fp32 partials through distributed shared memory and add them; IEEE
+//     operand), swap the fp32 partials through distributed shared memory (st.async into the
+//     peer's double-buffered inbox, completing on the peer's own mbarrier) and add them; IEEE
 //     addition commutes, so both hold bit-identical S and take identical softmax decisions;
 //   * each CTA accumulates P . V for its own 256 latent dims in TMEM (256 columns).
 // TMEM columns: O [0,256), S [256,320), P [320,352) (bf16 pairs), Q [352,496) (bf16 pairs).
@@ -41,7 +42,8 @@ constexpr int kStages = 4;
 constexpr int kSlabBytes = kRows * 64 * 2;                // 64 rows x 64 dims bf16: 8 KB
 constexpr int kRopeBytes = kRows * 32 * 2;                // 64 rows x 32 dims bf16: 4 KB
 constexpr int kStageBytes = 4 * kSlabBytes + kRopeBytes;  // 36 KB
-constexpr int kInboxBytes = kH * kRows * 4;               // 128 x 64 fp32: 32 KB
+constexpr int kInboxBytes = kH * kRows * 4;               // 128 x 64 fp32: 32 KB per slot
+constexpr int kInboxSlots = 2;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352;
@@ -51,9 +53,9 @@ enum Bar {
   kFull = 0,
   kEmpty = kFull + kStages,
   kSFull = kEmpty + kStages,
-  kSFree, kPFull, kPvDone, kQFull, kOFree, kXFull, kXFree, kFinal, kNumBars
+  kSFree, kPFull, kPvDone, kQFull, kOFree, kXFull, kFinal = kXFull + kInboxSlots, kNumBars
 };
-constexpr int kBarOff = kStages * kStageBytes + kInboxBytes;
+constexpr int kBarOff = kStages * kStageBytes + kInboxSlots * kInboxBytes;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // +1024: manual alignment
 
 // instruction descriptors, kind::f16: bf16 A and B, fp32 D, A K-major
@@ -97,23 +99,19 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void mbar_arrive_peer(uint32_t bar_in_peer) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_in_peer)
-               : "memory");
+// 16 bytes into the peer CTA's shared memory; completes bytes on the peer's mbarrier.
+__device__ __forceinline__ void st_async_peer(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                              uint32_t d, uint32_t peer_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(peer_bar)
+      : "memory");
 }
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;"
-      "\n\tselp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
   return ok != 0;
 }
@@ -158,6 +156,27 @@ __device__ __forceinline__ void tmem_ld32(uint32_t ta, uint32_t (&v)[32]) {
         "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
         "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(ta)
+      : "memory");
+}
+// 64 consecutive columns, one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t ta, uint32_t (&v)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,"
+      "%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
+        "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
+        "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31]), "=r"(v[32]), "=r"(v[33]), "=r"(v[34]),
+        "=r"(v[35]), "=r"(v[36]), "=r"(v[37]), "=r"(v[38]), "=r"(v[39]), "=r"(v[40]), "=r"(v[41]),
+        "=r"(v[42]), "=r"(v[43]), "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47]), "=r"(v[48]),
+        "=r"(v[49]), "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]), "=r"(v[55]),
+        "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]), "=r"(v[61]), "=r"(v[62]),
+        "=r"(v[63])
+      : "r"(ta), "r"(ta + 32u)
       : "memory");
 }
 __device__ __forceinline__ void tmem_st32(uint32_t ta, const uint32_t (&v)[32]) {
@@ -206,11 +225,10 @@ struct Ctl {
 };
 
 // Warp-collective bounded wait; the result is the same in all 32 lanes.
-__device__ __noinline__ bool warp_wait(uint32_t bar, uint32_t parity, bool cluster_scope,
-                                       const Ctl& c) {
+__device__ __noinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Ctl& c) {
   uint64_t t0 = 0;
   for (int it = 0;; ++it) {
-    const bool done = cluster_scope ? mbar_try_cluster(bar, parity) : mbar_try(bar, parity);
+    const bool done = mbar_try(bar, parity);
     if (__all_sync(0xffffffffu, done)) return true;
     if (it == 0) t0 = globaltimer();
     const bool late = (globaltimer() - t0) > kTimeoutNs;
@@ -224,12 +242,6 @@ __device__ __noinline__ bool warp_wait(uint32_t bar, uint32_t parity, bool clust
     }
   }
 }
-
-// Where a work range's tiles come from.
-struct TileInfo {
-  int bt, b, local, valid, slot;
-  bool first, last;
-};
 
 }  // namespace
 
@@ -261,9 +273,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
     mbar_init(bar(kPvDone), 1);
     mbar_init(bar(kQFull), 4);
     mbar_init(bar(kOFree), 4);
-    mbar_init(bar(kXFull), 128);
-    mbar_init(bar(kXFree), 128);
+    for (int i = 0; i < kInboxSlots; ++i) mbar_init(bar(kXFull + i), 1);
     mbar_init(bar(kFinal), 1);
+    // each inbox slot expects one partial score tile (from the peer) per phase
+    for (int i = 0; i < kInboxSlots; ++i) mbar_expect_tx(bar(kXFull + i), kInboxBytes);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -277,7 +290,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
   tc_before();
   __syncthreads();
   tc_after();
-  cluster_sync();  // barriers of both CTAs initialised before any remote arrive
+  cluster_sync();  // barriers of both CTAs initialised before any remote store
   const uint32_t tmem = *tmem_slot;
 
   // this pair's segments
@@ -288,70 +301,63 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
     se = p.range_begin[q + 1];
   }
 
-  // walks tiles in order; returns false at the end
-  auto tile_at = [&](int& s, int& c, TileInfo& ti) -> bool {
-    while (s < se) {
-      const Segment sg = p.segments[s];
-      if (c < sg.chunk_lo) c = sg.chunk_lo;
-      if (c < sg.chunk_hi) {
-        const int chunk0 = p.bt_chunk0[sg.bt];
-        ti.bt = sg.bt;
-        ti.b = sg.bt / p.T;
-        ti.local = c - chunk0;
-        ti.valid = min(kRows, p.bt_len[sg.bt] - ti.local * kRows);
-        ti.slot = sg.slot;
-        ti.first = (c == sg.chunk_lo);
-        ti.last = (c == sg.chunk_hi - 1);
-        return true;
-      }
-      ++s;
-      c = -1;
-    }
-    return false;
-  };
-
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    int s = sb, c = -1, t = 0;
-    TileInfo ti;
-    while (tile_at(s, c, ti)) {
-      const int stage = t % kStages;
-      if (t >= kStages && !warp_wait(bar(kEmpty + stage), ((t / kStages) - 1) & 1, false, ctl))
-        break;
-      if (lane == 0) {
-        int blk = p.table[(size_t)ti.b * p.max_blocks + ti.local];
-        if (blk < 0 || blk >= p.num_blocks) {
-          set_error(p.err, MLA_DEV_OOB_BLOCK);
-          blk = 0;
+    int t = 0;
+    bool ok = true;
+    for (int s = sb; ok && s < se; ++s) {
+      const Segment sg = p.segments[s];
+      const int b = sg.bt / p.T;
+      const int n = sg.chunk_hi - sg.chunk_lo;
+      const int32_t* trow =
+          p.table + (size_t)b * p.max_blocks + (sg.chunk_lo - p.bt_chunk0[sg.bt]);
+      for (int base = 0; ok && base < n; base += 32) {
+        // block ids of the next 32 chunks, one per lane
+        int my = 0;
+        if (base + lane < n) {
+          my = trow[base + lane];
+          if (my < 0 || my >= p.num_blocks) {
+            set_error(p.err, MLA_DEV_OOB_BLOCK);
+            my = 0;
+          }
         }
-        const uint32_t dst = s_base + stage * kStageBytes;
-        const uint32_t fb = bar(kFull + stage);
-        mbar_expect_tx(fb, kStageBytes);
-        for (int i = 0; i < 4; ++i)
-          tma_load(dst + i * kSlabBytes, &tm_ckv, fb, 256 * (int)rank + 64 * i, blk * kRows);
-        tma_load(dst + 4 * kSlabBytes, &tm_rope, fb, kR + 32 * (int)rank, blk * kRows);
+        const int cnt = min(32, n - base);
+        for (int i = 0; i < cnt; ++i) {
+          const int blk = __shfl_sync(0xffffffffu, my, i);
+          const int stage = t % kStages;
+          if (t >= kStages && !warp_wait(bar(kEmpty + stage), ((t / kStages) - 1) & 1, ctl)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            const uint32_t dst = s_base + stage * kStageBytes;
+            const uint32_t fb = bar(kFull + stage);
+            mbar_expect_tx(fb, kStageBytes);
+            for (int k = 0; k < 4; ++k)
+              tma_load(dst + k * kSlabBytes, &tm_ckv, fb, 256 * (int)rank + 64 * k, blk * kRows);
+            tma_load(dst + 4 * kSlabBytes, &tm_rope, fb, kR + 32 * (int)rank, blk * kRows);
+          }
+          __syncwarp();
+          ++t;
+        }
       }
-      __syncwarp();
-      ++t;
-      ++c;
     }
     // drain: every issued load has landed before the CTA may exit
     for (int k = 1; k <= kStages && k <= t; ++k) {
       const int tt = t - k;
-      uint64_t t0 = globaltimer();
+      const uint64_t t0 = globaltimer();
       bool done = false;
       while (!done && globaltimer() - t0 < kTimeoutNs)
         done = __all_sync(0xffffffffu, mbar_try(bar(kFull + tt % kStages), (tt / kStages) & 1));
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    int s = sb, c = -1, t = 0, seg_i = -1;
-    TileInfo ti;
+    int t = 0, seg_i = 0;
     int prev_stage = 0, prev_seg = 0;
     bool prev_first = false, have_prev = false, ok = true;
     auto issue_pv = [&](int tp) -> bool {
-      if (!warp_wait(bar(kPFull), tp & 1, false, ctl)) return false;
-      if (prev_first && prev_seg > 0 && !warp_wait(bar(kOFree), (prev_seg - 1) & 1, false, ctl))
+      if (!warp_wait(bar(kPFull), tp & 1, ctl)) return false;
+      if (prev_first && prev_seg > 0 && !warp_wait(bar(kOFree), (prev_seg - 1) & 1, ctl))
         return false;
       tc_after();
       if (lane == 0) {
@@ -366,46 +372,54 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
       __syncwarp();
       return true;
     };
-    while (ok && tile_at(s, c, ti)) {
-      const int stage = t % kStages;
-      if (ti.first) ++seg_i;
-      ok = warp_wait(bar(kFull + stage), (t / kStages) & 1, false, ctl);
-      if (ok && ti.first) ok = warp_wait(bar(kQFull), seg_i & 1, false, ctl);
-      if (ok && t > 0) ok = warp_wait(bar(kSFree), (t - 1) & 1, false, ctl);
-      if (!ok) break;
-      const uint32_t kbase = s_base + stage * kStageBytes;
-      if (ti.valid < kRows) {
-        // rows past the sequence end: zero their latent part so 0 * garbage never enters P . V
-        uint8_t* st = smem + stage * kStageBytes;
-        const int n16 = (kRows - ti.valid) * 128 / 16;
-        for (int slab = 0; slab < 4; ++slab) {
-          uint4* z = (uint4*)(st + slab * kSlabBytes + ti.valid * 128);
-          for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
+    for (int s = sb; ok && s < se; ++s, ++seg_i) {
+      const Segment sg = p.segments[s];
+      const int chunk0 = p.bt_chunk0[sg.bt];
+      const int len = p.bt_len[sg.bt];
+      for (int c = sg.chunk_lo; c < sg.chunk_hi; ++c) {
+        const bool first = (c == sg.chunk_lo);
+        const int valid = min(kRows, len - (c - chunk0) * kRows);
+        const int stage = t % kStages;
+        ok = warp_wait(bar(kFull + stage), (t / kStages) & 1, ctl);
+        if (ok && first) ok = warp_wait(bar(kQFull), seg_i & 1, ctl);
+        if (ok && t > 0) ok = warp_wait(bar(kSFree), (t - 1) & 1, ctl);
+        if (!ok) break;
+        const uint32_t kbase = s_base + stage * kStageBytes;
+        if (valid < kRows) {
+          // rows past the sequence end: zero their latent part so 0 * garbage never enters P . V
+          uint8_t* st = smem + stage * kStageBytes;
+          const int n16 = (kRows - valid) * 128 / 16;
+          for (int slab = 0; slab < 4; ++slab) {
+            uint4* z = (uint4*)(st + slab * kSlabBytes + valid * 128);
+            for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async();
+          __syncwarp();
         }
-        fence_proxy_async();
+        tc_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k)  // latent half: four 64-dim slabs, 16 dims per step
+            mma_ts(tmem + kColS, tmem + kColQ + 8 * k,
+                   sdesc(kbase + (k >> 2) * kSlabBytes + (k & 3) * 32, 16, 1024, 2), kIdescQK,
+                   k > 0 ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 2; ++k)  // RoPE half: 32 dims, 64-byte swizzle
+            mma_ts(tmem + kColS, tmem + kColQ + 128 + 8 * k,
+                   sdesc(kbase + 4 * kSlabBytes + k * 32, 16, 512, 4), kIdescQK, 1u);
+          tc_commit(bar(kSFull));
+        }
         __syncwarp();
+        if (have_prev && !issue_pv(t - 1)) {
+          ok = false;
+          break;
+        }
+        prev_stage = stage;
+        prev_first = first;
+        prev_seg = seg_i;
+        have_prev = true;
+        ++t;
       }
-      tc_after();
-      if (lane == 0) {
-#pragma unroll
-        for (int k = 0; k < 16; ++k)  // latent half: four 64-dim slabs, 16 dims per step
-          mma_ts(tmem + kColS, tmem + kColQ + 8 * k,
-                 sdesc(kbase + (k >> 2) * kSlabBytes + (k & 3) * 32, 16, 1024, 2), kIdescQK,
-                 k > 0 ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 2; ++k)  // RoPE half: 32 dims, 64-byte swizzle
-          mma_ts(tmem + kColS, tmem + kColQ + 128 + 8 * k,
-                 sdesc(kbase + 4 * kSlabBytes + k * 32, 16, 512, 4), kIdescQK, 1u);
-        tc_commit(bar(kSFull));
-      }
-      __syncwarp();
-      if (have_prev && !issue_pv(t - 1)) { ok = false; break; }
-      prev_stage = stage;
-      prev_first = ti.first;
-      prev_seg = seg_i;
-      have_prev = true;
-      ++t;
-      ++c;
     }
     if (ok && have_prev) issue_pv(t - 1);
   } else {
@@ -415,10 +429,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const float c2 = p.scale * 1.4426950408889634f;  // scores in log2 units
     const __nv_bfloat16* Q = (const __nv_bfloat16*)p.q;
-    const uint32_t my_row = s_inbox + (uint32_t)h * (kRows * 4);
-    const uint32_t peer_row = peer_addr(my_row, peer);
-    const uint32_t peer_xfull = peer_addr(bar(kXFull), peer);
-    const uint32_t peer_xfree = peer_addr(bar(kXFree), peer);
+    const uint32_t row_off = (uint32_t)h * (kRows * 4);
+    const uint32_t peer_inbox = peer_addr(s_inbox, peer);
+    uint32_t peer_xfull[kInboxSlots];
+#pragma unroll
+    for (int i = 0; i < kInboxSlots; ++i) peer_xfull[i] = peer_addr(bar(kXFull + i), peer);
     const int swz = h & 15;
 
     auto load_q = [&](int bt) {
@@ -446,142 +461,136 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
       if (lane == 0) mbar_arrive(bar(kQFull));
     };
 
-    int s = sb, c = -1, t = 0;
-    TileInfo ti;
+    int t = 0;
     float m_ref = 0.f, l = 0.f;
-    bool ok = true, q_loaded = false;
-    while (ok && tile_at(s, c, ti)) {
-      if (!q_loaded) {  // first segment of the range
-        load_q(ti.bt);
-        q_loaded = true;
-      }
-      // own partial scores
-      if (!warp_wait(bar(kSFull), t & 1, false, ctl)) { ok = false; break; }
-      tc_after();
-      uint32_t sv[64];
-      {
-        uint32_t a[32], b2[32];
-        tmem_ld32(tl + kColS, a);
-        tmem_ld32(tl + kColS + 32, b2);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) { sv[i] = a[i]; sv[32 + i] = b2[i]; }
-      }
-      tc_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kSFree));
+    bool ok = true;
+    if (sb < se) load_q(p.segments[sb].bt);
+    for (int s = sb; ok && s < se; ++s) {
+      const Segment sg = p.segments[s];
+      const int chunk0 = p.bt_chunk0[sg.bt];
+      const int len = p.bt_len[sg.bt];
+      for (int c = sg.chunk_lo; ok && c < sg.chunk_hi; ++c) {
+        const bool first = (c == sg.chunk_lo), last = (c == sg.chunk_hi - 1);
+        const int valid = min(kRows, len - (c - chunk0) * kRows);
 
-      // swap partials with the other CTA of the pair
-      if (t > 0 && !warp_wait(bar(kXFree), (t - 1) & 1, true, ctl)) { ok = false; break; }
-#pragma unroll
-      for (int u = 0; u < 16; ++u)
-        asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                         peer_row + 16u * (uint32_t)(u ^ swz)),
-                     "r"(sv[4 * u]), "r"(sv[4 * u + 1]), "r"(sv[4 * u + 2]), "r"(sv[4 * u + 3])
-                     : "memory");
-      mbar_arrive_peer(peer_xfull);
-      if (!warp_wait(bar(kXFull), t & 1, true, ctl)) { ok = false; break; }
-      float x[64];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        uint4 v;
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                     : "r"(my_row + 16u * (uint32_t)(u ^ swz))
-                     : "memory");
-        x[4 * u] = __uint_as_float(sv[4 * u]) + __uint_as_float(v.x);
-        x[4 * u + 1] = __uint_as_float(sv[4 * u + 1]) + __uint_as_float(v.y);
-        x[4 * u + 2] = __uint_as_float(sv[4 * u + 2]) + __uint_as_float(v.z);
-        x[4 * u + 3] = __uint_as_float(sv[4 * u + 3]) + __uint_as_float(v.w);
-      }
-      mbar_arrive_peer(peer_xfree);
-
-      // online softmax in log2 units, lazy rescale of O
-      float mt = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        x[k] = (k < ti.valid) ? x[k] * c2 : -INFINITY;
-        mt = fmaxf(mt, x[k]);
-      }
-      float alpha = 1.f;
-      bool rescale = false;
-      if (ti.first) {
-        m_ref = mt;
-        l = 0.f;
-      } else if (mt > m_ref + 8.f) {
-        alpha = ex2(m_ref - mt);
-        m_ref = mt;
-        rescale = true;
-      }
-      float rs = 0.f;
-      uint32_t pw[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float p0 = ex2(x[2 * k] - m_ref);
-        const float p1 = ex2(x[2 * k + 1] - m_ref);
-        rs += p0;
-        rs += p1;
-        pw[k] = pack_bf16(p0, p1);
-      }
-      l = l * alpha + rs;
-
-      // P . V of the previous tile must be done before P and O are touched
-      if (t > 0 && !warp_wait(bar(kPvDone), (t - 1) & 1, false, ctl)) { ok = false; break; }
-      tc_after();
-      if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(tl + kColO + 32 * ch, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tl + kColO + 32 * ch, o);
-        }
-      }
-      tmem_st32(tl + kColP, pw);
-      tmem_wait_st();
-      tc_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kPFull));
-      ++t;
-
-      if (ti.last) {
-        // next segment's query goes in while this segment drains
-        {
-          int s2 = s, c2i = c + 1;
-          TileInfo nx;
-          if (tile_at(s2, c2i, nx)) load_q(nx.bt);
-        }
-        if (!warp_wait(bar(kPvDone), (t - 1) & 1, false, ctl)) { ok = false; break; }
+        // own partial scores
+        if (!warp_wait(bar(kSFull), t & 1, ctl)) { ok = false; break; }
         tc_after();
-        const float inv_l = 1.f / l;
-        const float lse = (m_ref + __log2f(l)) * 0.6931471805599453f;
-        float* dst = (ti.slot < 0 ? p.out + ((size_t)ti.bt * kH + h) * kR
-                                  : p.part_o + ((size_t)ti.slot * kH + h) * kR) +
-                     256 * rank;
-#pragma unroll 1
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(tl + kColO + 32 * ch, o);
-          float4* d4 = (float4*)(dst + 32 * ch);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l,
-                                __uint_as_float(o[4 * i + 1]) * inv_l,
-                                __uint_as_float(o[4 * i + 2]) * inv_l,
-                                __uint_as_float(o[4 * i + 3]) * inv_l);
-        }
-        if (rank == 0) {
-          if (ti.slot < 0) {
-            if (p.lse) p.lse[(size_t)ti.bt * kH + h] = lse;
-          } else {
-            p.part_lse[(size_t)ti.slot * kH + h] = lse;
-          }
-        }
+        uint32_t sv[64];
+        tmem_ld64(tl + kColS, sv);
         tc_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kOFree));
+        if (lane == 0) mbar_arrive(bar(kSFree));
+
+        // swap partials with the other CTA: write into its inbox slot, read ours
+        const int slot = t & 1;
+        const uint32_t pdst = peer_inbox + (uint32_t)slot * kInboxBytes + row_off;
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          st_async_peer(pdst + 16u * (uint32_t)(u ^ swz), sv[4 * u], sv[4 * u + 1], sv[4 * u + 2],
+                        sv[4 * u + 3], peer_xfull[slot]);
+        if (!warp_wait(bar(kXFull + slot), (t >> 1) & 1, ctl)) { ok = false; break; }
+        float x[64];
+        const uint32_t mine = s_inbox + (uint32_t)slot * kInboxBytes + row_off;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          uint4 v;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(mine + 16u * (uint32_t)(u ^ swz))
+                       : "memory");
+          x[4 * u] = __uint_as_float(sv[4 * u]) + __uint_as_float(v.x);
+          x[4 * u + 1] = __uint_as_float(sv[4 * u + 1]) + __uint_as_float(v.y);
+          x[4 * u + 2] = __uint_as_float(sv[4 * u + 2]) + __uint_as_float(v.z);
+          x[4 * u + 3] = __uint_as_float(sv[4 * u + 3]) + __uint_as_float(v.w);
+        }
+        // this slot's next use is tile t + 2; the peer can only write it after receiving our
+        // partial of tile t + 1, so re-arming now cannot race with this tile's reads
+        if (threadIdx.x == 64) mbar_expect_tx(bar(kXFull + slot), kInboxBytes);
+
+        // online softmax in log2 units, lazy rescale of O
+        float mt = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          x[k] = (k < valid) ? x[k] * c2 : -INFINITY;
+          mt = fmaxf(mt, x[k]);
+        }
+        float alpha = 1.f;
+        bool rescale = false;
+        if (first) {
+          m_ref = mt;
+          l = 0.f;
+        } else if (mt > m_ref + 8.f) {
+          alpha = ex2(m_ref - mt);
+          m_ref = mt;
+          rescale = true;
+        }
+        float rs = 0.f;
+        uint32_t pw[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float p0 = ex2(x[2 * k] - m_ref);
+          const float p1 = ex2(x[2 * k + 1] - m_ref);
+          rs += p0;
+          rs += p1;
+          pw[k] = pack_bf16(p0, p1);
+        }
+        l = l * alpha + rs;
+
+        // P . V of the previous tile must be done before P and O are touched
+        if (t > 0 && !warp_wait(bar(kPvDone), (t - 1) & 1, ctl)) { ok = false; break; }
+        tc_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+          for (int ch = 0; ch < 8; ++ch) {
+            uint32_t o[32];
+            tmem_ld32(tl + kColO + 32 * ch, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tl + kColO + 32 * ch, o);
+          }
+        }
+        tmem_st32(tl + kColP, pw);
+        tmem_wait_st();
+        tc_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kPFull));
+        ++t;
+
+        if (last) {
+          // next segment's query goes in while this segment drains
+          if (s + 1 < se) load_q(p.segments[s + 1].bt);
+          if (!warp_wait(bar(kPvDone), (t - 1) & 1, ctl)) { ok = false; break; }
+          tc_after();
+          const float inv_l = 1.f / l;
+          const float lse = (m_ref + __log2f(l)) * 0.6931471805599453f;
+          float* dst = (sg.slot < 0 ? p.out + ((size_t)sg.bt * kH + h) * kR
+                                    : p.part_o + ((size_t)sg.slot * kH + h) * kR) +
+                       256 * rank;
+#pragma unroll 1
+          for (int ch = 0; ch < 8; ++ch) {
+            uint32_t o[32];
+            tmem_ld32(tl + kColO + 32 * ch, o);
+            float4* d4 = (float4*)(dst + 32 * ch);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              d4[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l,
+                                  __uint_as_float(o[4 * i + 1]) * inv_l,
+                                  __uint_as_float(o[4 * i + 2]) * inv_l,
+                                  __uint_as_float(o[4 * i + 3]) * inv_l);
+          }
+          if (rank == 0) {
+            if (sg.slot < 0) {
+              if (p.lse) p.lse[(size_t)sg.bt * kH + h] = lse;
+            } else {
+              p.part_lse[(size_t)sg.slot * kH + h] = lse;
+            }
+          }
+          tc_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kOFree));
+        }
       }
-      ++c;
     }
   }
 
@@ -592,7 +601,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
   if (warp == 1) {
     if (lane == 0) tc_commit(bar(kFinal));  // completes once every MMA issued here is done
     __syncwarp();
-    uint64_t t0 = globaltimer();
+    const uint64_t t0 = globaltimer();
     bool done = false;
     while (!done && globaltimer() - t0 < kTimeoutNs)
       done = __all_sync(0xffffffffu, mbar_try(bar(kFinal), 0));
