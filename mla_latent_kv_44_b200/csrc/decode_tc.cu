@@ -4,27 +4,26 @@
 // Absorbed decode ("DeepSeek MLA, Built From the Paper", 3 Matrix absorption; "Build a DeepSeek
 // Model from Scratch" ch. 3, score = content score + position score; "MLA from scratch in
 // PyTorch", Absorbing projections: attend directly to latents). For one query token the 128
-// heads are the M = 128 rows of two dense contractions against the shared cache tile:
-//   S = Q . K^T      (M = 128 heads, N = 64 rows, K = 576 = [c_kv || k_rope])
-//   O += P . V       (M = 128 heads, N = 512 latent dims, K = 64 rows; V = the c_kv part of K)
-// so each cache tile is read from HBM once and serves both products.
+// heads are the M = 128 rows of two dense contractions against the shared cache rows:
+//   S = Q . K^T      (M = 128 heads, N = rows, K = 576 = [c_kv || k_rope])
+//   O += P . V       (M = 128 heads, N = 512 latent dims, K = rows; V = the c_kv part of K)
 //
-// O for 128 heads x 512 dims in fp32 is 256 KB: all of one SM's tensor memory. A cluster of two
-// CTAs therefore shares every work range. CTA c loads only its half of each row -- latent dims
-// [256c, 256c + 256) and RoPE dims [32c, 32c + 32) -- so the pair reads each cache byte once:
-//   * both CTAs compute a partial S over their 288 dims (Q half resident in TMEM as the A
-//     operand), swap the fp32 partials through distributed shared memory (st.async into the
-//     peer's double-buffered inbox, completing on the peer's own mbarrier) and add them; IEEE
-//     addition commutes, so both hold bit-identical S and take identical softmax decisions;
-//   * each CTA accumulates P . V for its own 256 latent dims in TMEM (256 columns).
-// TMEM columns: O [0,256), S [256,320), P [320,352) (bf16 pairs), Q [352,496) (bf16 pairs).
-//
-// Warp roles: warp 0 issues TMA loads into a 4-stage ring, warp 1 issues the MMAs (QK of tile
-// t+1 before PV of tile t, so the tensor pipe works while the softmax warps work), warps 2-5
-// (one TMEM lane per head) run the online softmax in exp2 units with a lazy rescale of O (only
-// when the running max grows by more than 2^8), and the epilogue. Every wait is bounded: on
-// timeout the kernel sets MLA_DEV_WAIT_TIMEOUT, drains its own copies and MMAs, frees TMEM and
-// returns. No TMA multicast is used.
+// A tcgen05.mma instruction costs about the same whatever its N (up to 256), so both products
+// are issued with N = 256: S over tiles of 256 rows (four 64-row cache blocks), O over 256
+// latent dims at a time. O for 128 heads x 512 dims in fp32 fills one SM's tensor memory, so
+// the two CTAs of a cluster take different roles for each work range:
+//   * the score CTA keeps the latent part of Q in TMEM (256 columns, A operand) and its RoPE
+//     part in shared memory, streams the cache rows' 64-dim slabs by TMA, accumulates S in the
+//     other 256 TMEM columns, runs the online softmax (exp2 units, O rescaled lazily only when
+//     the running max grows by more than 2^8) and sends P (bf16) with the per-row rescale
+//     factors and sums to the value CTA as 16 KB bulk copies into a 6-slot ring in its shared
+//     memory;
+//   * the value CTA streams the latent part of the same rows by TMA and accumulates O = P . V
+//     in its whole TMEM, applies rescales, and writes the normalised output.
+// The two read the same cache blocks close together in time, so HBM sees each row about once.
+// Warps: 0 TMA, 1 MMA issue, 2-5 softmax (score CTA) or rescale and epilogue (value CTA).
+// Every wait is bounded: on timeout the kernel sets MLA_DEV_WAIT_TIMEOUT, drains its copies
+// and MMAs, frees TMEM and returns. No TMA multicast is used.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -37,33 +36,64 @@ constexpr int kH = 128;
 constexpr int kR = 512;
 constexpr int kDR = 64;
 constexpr int kD = kR + kDR;
-constexpr int kRows = 64;                                 // rows per tile = block = chunk
-constexpr int kStages = 4;
-constexpr int kSlabBytes = kRows * 64 * 2;                // 64 rows x 64 dims bf16: 8 KB
-constexpr int kRopeBytes = kRows * 32 * 2;                // 64 rows x 32 dims bf16: 4 KB
-constexpr int kStageBytes = 4 * kSlabBytes + kRopeBytes;  // 36 KB
-constexpr int kInboxBytes = kH * kRows * 4;               // 128 x 64 fp32: 32 KB per slot
-constexpr int kInboxSlots = 2;
+constexpr int kRows = 64;                       // rows per cache block = planner chunk
+constexpr int kTileBlocks = 4;                  // blocks per score tile (N <= 256)
+constexpr int kSlabBytes = kRows * 64 * 2;      // 64 rows x 64 dims bf16: 8 KB
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352;
 constexpr unsigned long long kTimeoutNs = 1000000000ull;  // 1 s per wait
 
+// score CTA: K stages of one 64-dim slab for up to four blocks, RoPE part of Q, P staging
+constexpr int kKStages = 4;
+constexpr int kKStageBytes = kTileBlocks * kSlabBytes;        // 32 KB
+constexpr int kQRopeBytes = kH * 64 * 2;                      // 16 KB
+constexpr int kPBlockBytes = kH * kRows * 2;                  // 128 x 64 bf16: 16 KB
+constexpr int kHdrBytes = 2 * kH * 4;                         // alpha[128], l[128]
+constexpr int kS_K = 0;
+constexpr int kS_QRope = kS_K + kKStages * kKStageBytes;      // 128 KB
+constexpr int kS_Stage = kS_QRope + kQRopeBytes;              // 144 KB
+constexpr int kS_Hdr = kS_Stage + kTileBlocks * kPBlockBytes; // 208 KB
+constexpr int kS_End = kS_Hdr + kHdrBytes;
+// value CTA: V stages (one block's 256-dim half), P ring, header ring
+constexpr int kVStages = 3;
+constexpr int kVStageBytes = 4 * kSlabBytes;                  // 32 KB
+constexpr int kPSlots = 6;
+constexpr int kHdrSlots = 2;
+constexpr int kV_V = 0;
+constexpr int kV_P = kV_V + kVStages * kVStageBytes;          // 96 KB
+constexpr int kV_Hdr = kV_P + kPSlots * kPBlockBytes;         // 192 KB
+constexpr int kV_End = kV_Hdr + kHdrSlots * kHdrBytes;
+constexpr int kDataBytes = kS_End > kV_End ? kS_End : kV_End;
+
 enum Bar {
-  kFull = 0,
-  kEmpty = kFull + kStages,
-  kSFull = kEmpty + kStages,
-  kSFree, kPFull, kPvDone, kQFull, kOFree, kXFull, kFinal = kXFull + kInboxSlots, kNumBars
+  // score CTA
+  kKFull = 0,
+  kKEmpty = kKFull + kKStages,
+  kQFull = kKEmpty + kKStages,  // Q of the segment in place (TMA RoPE part + 4 softmax warps)
+  kQEmpty,                      // last S product of the segment done with Q
+  kSFull,                       // S complete
+  kSFree,                       // softmax done reading S
+  kStgFree,                     // value CTA received the previous tile's P (staging reusable)
+  kSlotFree,                    // kPSlots: value CTA finished with a P ring slot
+  // value CTA
+  kVFull = kSlotFree + kPSlots,
+  kVEmpty = kVFull + kVStages,
+  kPFull = kVEmpty + kVStages,  // kPSlots
+  kHFull = kPFull + kPSlots,    // kHdrSlots
+  kSlotDone = kHFull + kHdrSlots,  // kPSlots: P . V MMAs reading a slot are complete
+  kOReady = kSlotDone + kPSlots,   // rescale (if any) applied, previous epilogue done
+  kPvDone,                         // 2: all P . V of a tile complete (even / odd tiles)
+  kFinal = kPvDone + 2,
+  kNumBars
 };
-constexpr int kBarOff = kStages * kStageBytes + kInboxSlots * kInboxBytes;
+constexpr int kBarOff = kDataBytes;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // +1024: manual alignment
 
 // instruction descriptors, kind::f16: bf16 A and B, fp32 D, A K-major
-constexpr uint32_t idesc(int M, int N, int b_mn_major) {
+__host__ __device__ constexpr uint32_t idesc(int M, int N, int b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-constexpr uint32_t kIdescQK = idesc(128, 64, 0);
 constexpr uint32_t kIdescPV = idesc(128, 256, 1);
 
 // ------------------------------------------------------------------------------ PTX helpers
@@ -98,14 +128,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// 16 bytes into the peer CTA's shared memory; completes bytes on the peer's mbarrier.
-__device__ __forceinline__ void st_async_peer(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                              uint32_t d, uint32_t peer_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
-      ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(peer_bar)
-      : "memory");
 }
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -190,14 +212,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t ta, const uint32_t (&v)[32]) 
       "r"(v[30]), "r"(v[31])
       : "memory");
 }
-__device__ __forceinline__ void tmem_st16(uint32_t ta, const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16};" ::"r"(ta),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-      : "memory");
-}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -217,6 +231,32 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
                                           uint32_t swz) {
   return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | ((uint64_t)swz << 61);
+}
+
+// D[tmem] (+)= A[smem] . B[smem]
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t id,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d), "l"(adesc),
+      "l"(bdesc), "r"(id), "r"(acc)
+      : "memory");
+}
+// shared::cta -> peer shared::cluster bulk copy, completing bytes on the peer's mbarrier
+__device__ __forceinline__ void bulk_to_peer(uint32_t dst, uint32_t src, uint32_t bytes,
+                                             uint32_t peer_bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "r"(src), "r"(bytes), "r"(peer_bar)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t bar_in_peer) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_in_peer)
+               : "memory");
+}
+// the four softmax / epilogue warps (threads 64..191)
+__device__ __forceinline__ void sync_math_warps() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
 struct Ctl {
@@ -243,15 +283,69 @@ __device__ __noinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Ctl&
   }
 }
 
+// Bounded wait for a phase that normally completed long ago (drains at teardown).
+__device__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
+  const uint64_t t0 = globaltimer();
+  bool done = false;
+  while (!done && globaltimer() - t0 < kTimeoutNs) done = __all_sync(0xffffffffu, mbar_try(bar, parity));
+  if (!done && (threadIdx.x & 31) == 0) set_error(err, MLA_DEV_WAIT_TIMEOUT);
+}
+
+// One score tile: up to four consecutive cache blocks of one segment.
+struct Tile {
+  int bt, b, local0, nb, ntok, slot;
+  bool first, last;
+};
+
+// Walks the tiles of segments [s, se) in order (identically in both CTAs).
+struct TileWalk {
+  const DecodeParams* p;
+  int s, se, c;  // current segment and chunk
+  __device__ bool next(Tile& tl) {
+    while (s < se) {
+      const Segment sg = p->segments[s];
+      if (c < sg.chunk_lo) c = sg.chunk_lo;
+      if (c < sg.chunk_hi) {
+        const int chunk0 = p->bt_chunk0[sg.bt];
+        tl.bt = sg.bt;
+        tl.b = sg.bt / p->T;
+        tl.local0 = c - chunk0;
+        tl.nb = min(kTileBlocks, sg.chunk_hi - c);
+        tl.ntok = min(tl.nb * kRows, p->bt_len[sg.bt] - tl.local0 * kRows);
+        tl.slot = sg.slot;
+        tl.first = (c == sg.chunk_lo);
+        tl.last = (c + tl.nb == sg.chunk_hi);
+        c += tl.nb;
+        return true;
+      }
+      ++s;
+      c = -1;
+    }
+    return false;
+  }
+};
+
+// Block ids of a tile (lane j < nb holds block j), out-of-pool ids flagged and replaced by 0.
+__device__ __forceinline__ int tile_block(const DecodeParams& p, const Tile& tl, int lane) {
+  int blk = 0;
+  if (lane < tl.nb) {
+    blk = p.table[(size_t)tl.b * p.max_blocks + tl.local0 + lane];
+    if (blk < 0 || blk >= p.num_blocks) {
+      set_error(p.err, MLA_DEV_OOB_BLOCK);
+      blk = 0;
+    }
+  }
+  return blk;
+}
+
 }  // namespace
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
-                 const __grid_constant__ CUtensorMap tm_rope, const DecodeParams p) {
+attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
+                 const __grid_constant__ CUtensorMap tm_q, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t s_base = saddr(smem);
-  const uint32_t s_inbox = s_base + kStages * kStageBytes;
   const uint32_t s_bar = s_base + kBarOff;
   uint32_t* tmem_slot = (uint32_t*)(smem + kBarOff + kNumBars * 8);
   volatile int* abort_flag = (volatile int*)(smem + kBarOff + kNumBars * 8 + 4);
@@ -260,23 +354,39 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const uint32_t peer = rank ^ 1u;
+  const bool score = (rank == 0);
   const Ctl ctl{p.err, abort_flag};
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(bar(kFull + i), 1);
-      mbar_init(bar(kEmpty + i), 1);
+    if (score) {
+      for (int i = 0; i < kKStages; ++i) {
+        mbar_init(bar(kKFull + i), 1);
+        mbar_init(bar(kKEmpty + i), 1);
+      }
+      mbar_init(bar(kQFull), 5);
+      mbar_init(bar(kQEmpty), 1);
+      mbar_init(bar(kSFull), 1);
+      mbar_init(bar(kSFree), 4);
+      mbar_init(bar(kStgFree), 1);
+      for (int i = 0; i < kPSlots; ++i) mbar_init(bar(kSlotFree + i), 1);
+    } else {
+      for (int i = 0; i < kVStages; ++i) {
+        mbar_init(bar(kVFull + i), 1);
+        mbar_init(bar(kVEmpty + i), 1);
+      }
+      for (int i = 0; i < kPSlots; ++i) {
+        mbar_init(bar(kPFull + i), 1);
+        mbar_init(bar(kSlotDone + i), 1);
+      }
+      for (int i = 0; i < kHdrSlots; ++i) mbar_init(bar(kHFull + i), 1);
+      mbar_init(bar(kOReady), 4);
+      mbar_init(bar(kPvDone), 1);
+      mbar_init(bar(kPvDone + 1), 1);
+      // every P slot and header slot expects one bulk copy from the score CTA per use
+      for (int i = 0; i < kPSlots; ++i) mbar_expect_tx(bar(kPFull + i), kPBlockBytes);
+      for (int i = 0; i < kHdrSlots; ++i) mbar_expect_tx(bar(kHFull + i), kHdrBytes);
     }
-    mbar_init(bar(kSFull), 1);
-    mbar_init(bar(kSFree), 4);
-    mbar_init(bar(kPFull), 4);
-    mbar_init(bar(kPvDone), 1);
-    mbar_init(bar(kQFull), 4);
-    mbar_init(bar(kOFree), 4);
-    for (int i = 0; i < kInboxSlots; ++i) mbar_init(bar(kXFull + i), 1);
     mbar_init(bar(kFinal), 1);
-    // each inbox slot expects one partial score tile (from the peer) per phase
-    for (int i = 0; i < kInboxSlots; ++i) mbar_expect_tx(bar(kXFull + i), kInboxBytes);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -290,307 +400,383 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
   tc_before();
   __syncthreads();
   tc_after();
-  cluster_sync();  // barriers of both CTAs initialised before any remote store
+  cluster_sync();  // barriers of both CTAs initialised before any remote traffic
   const uint32_t tmem = *tmem_slot;
 
-  // this pair's segments
   const int q = blockIdx.x >> 1;
   int sb = 0, se = 0;
   if (q < p.header[1]) {
     sb = p.range_begin[q];
     se = p.range_begin[q + 1];
   }
+  TileWalk walk{&p, sb, se, -1};
+  Tile tl;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    int t = 0;
+  if (score && warp == 0) {
+    // ---------------------------------------------------------------- score: TMA producer
+    int kt = 0, seg_i = 0;
     bool ok = true;
-    for (int s = sb; ok && s < se; ++s) {
-      const Segment sg = p.segments[s];
-      const int b = sg.bt / p.T;
-      const int n = sg.chunk_hi - sg.chunk_lo;
-      const int32_t* trow =
-          p.table + (size_t)b * p.max_blocks + (sg.chunk_lo - p.bt_chunk0[sg.bt]);
-      for (int base = 0; ok && base < n; base += 32) {
-        // block ids of the next 32 chunks, one per lane
-        int my = 0;
-        if (base + lane < n) {
-          my = trow[base + lane];
-          if (my < 0 || my >= p.num_blocks) {
-            set_error(p.err, MLA_DEV_OOB_BLOCK);
-            my = 0;
-          }
-        }
-        const int cnt = min(32, n - base);
-        for (int i = 0; i < cnt; ++i) {
-          const int blk = __shfl_sync(0xffffffffu, my, i);
-          const int stage = t % kStages;
-          if (t >= kStages && !warp_wait(bar(kEmpty + stage), ((t / kStages) - 1) & 1, ctl)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) {
-            const uint32_t dst = s_base + stage * kStageBytes;
-            const uint32_t fb = bar(kFull + stage);
-            mbar_expect_tx(fb, kStageBytes);
-            for (int k = 0; k < 4; ++k)
-              tma_load(dst + k * kSlabBytes, &tm_ckv, fb, 256 * (int)rank + 64 * k, blk * kRows);
-            tma_load(dst + 4 * kSlabBytes, &tm_rope, fb, kR + 32 * (int)rank, blk * kRows);
-          }
-          __syncwarp();
-          ++t;
-        }
-      }
-    }
-    // drain: every issued load has landed before the CTA may exit
-    for (int k = 1; k <= kStages && k <= t; ++k) {
-      const int tt = t - k;
-      const uint64_t t0 = globaltimer();
-      bool done = false;
-      while (!done && globaltimer() - t0 < kTimeoutNs)
-        done = __all_sync(0xffffffffu, mbar_try(bar(kFull + tt % kStages), (tt / kStages) & 1));
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    int t = 0, seg_i = 0;
-    int prev_stage = 0, prev_seg = 0;
-    bool prev_first = false, have_prev = false, ok = true;
-    auto issue_pv = [&](int tp) -> bool {
-      if (!warp_wait(bar(kPFull), tp & 1, ctl)) return false;
-      if (prev_first && prev_seg > 0 && !warp_wait(bar(kOFree), (prev_seg - 1) & 1, ctl))
-        return false;
-      tc_after();
-      if (lane == 0) {
-        const uint32_t vbase = s_base + prev_stage * kStageBytes;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)  // 16 rows per step; MN-major B: LBO = 64-dim slab, SBO = 8 rows
-          mma_ts(tmem + kColO, tmem + kColP + 8 * k, sdesc(vbase + k * 2048, kSlabBytes, 1024, 2),
-                 kIdescPV, (prev_first && k == 0) ? 0u : 1u);
-        tc_commit(bar(kPvDone));
-        tc_commit(bar(kEmpty + prev_stage));
-      }
-      __syncwarp();
-      return true;
-    };
-    for (int s = sb; ok && s < se; ++s, ++seg_i) {
-      const Segment sg = p.segments[s];
-      const int chunk0 = p.bt_chunk0[sg.bt];
-      const int len = p.bt_len[sg.bt];
-      for (int c = sg.chunk_lo; c < sg.chunk_hi; ++c) {
-        const bool first = (c == sg.chunk_lo);
-        const int valid = min(kRows, len - (c - chunk0) * kRows);
-        const int stage = t % kStages;
-        ok = warp_wait(bar(kFull + stage), (t / kStages) & 1, ctl);
-        if (ok && first) ok = warp_wait(bar(kQFull), seg_i & 1, ctl);
-        if (ok && t > 0) ok = warp_wait(bar(kSFree), (t - 1) & 1, ctl);
-        if (!ok) break;
-        const uint32_t kbase = s_base + stage * kStageBytes;
-        if (valid < kRows) {
-          // rows past the sequence end: zero their latent part so 0 * garbage never enters P . V
-          uint8_t* st = smem + stage * kStageBytes;
-          const int n16 = (kRows - valid) * 128 / 16;
-          for (int slab = 0; slab < 4; ++slab) {
-            uint4* z = (uint4*)(st + slab * kSlabBytes + valid * 128);
-            for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async();
-          __syncwarp();
-        }
-        tc_after();
+    while (ok && walk.next(tl)) {
+      if (tl.first) {  // RoPE part of Q for this segment, once the previous segment's S is done
+        if (seg_i > 0 && !warp_wait(bar(kQEmpty), (seg_i - 1) & 1, ctl)) break;
         if (lane == 0) {
-#pragma unroll
-          for (int k = 0; k < 16; ++k)  // latent half: four 64-dim slabs, 16 dims per step
-            mma_ts(tmem + kColS, tmem + kColQ + 8 * k,
-                   sdesc(kbase + (k >> 2) * kSlabBytes + (k & 3) * 32, 16, 1024, 2), kIdescQK,
-                   k > 0 ? 1u : 0u);
-#pragma unroll
-          for (int k = 0; k < 2; ++k)  // RoPE half: 32 dims, 64-byte swizzle
-            mma_ts(tmem + kColS, tmem + kColQ + 128 + 8 * k,
-                   sdesc(kbase + 4 * kSlabBytes + k * 32, 16, 512, 4), kIdescQK, 1u);
-          tc_commit(bar(kSFull));
+          mbar_expect_tx(bar(kQFull), kQRopeBytes);
+          tma_load(s_base + kS_QRope, &tm_q, bar(kQFull), kR, tl.bt * kH);
         }
         __syncwarp();
-        if (have_prev && !issue_pv(t - 1)) {
+        ++seg_i;
+      }
+      const int my_blk = tile_block(p, tl, lane);
+      for (int k = 0; k < 9 && ok; ++k, ++kt) {  // 8 latent slabs, then the RoPE slab
+        const int stage = kt % kKStages;
+        if (kt >= kKStages && !warp_wait(bar(kKEmpty + stage), ((kt / kKStages) - 1) & 1, ctl)) {
           ok = false;
           break;
         }
-        prev_stage = stage;
-        prev_first = first;
-        prev_seg = seg_i;
-        have_prev = true;
-        ++t;
+        if (lane == 0) mbar_expect_tx(bar(kKFull + stage), tl.nb * kSlabBytes);
+        for (int j = 0; j < tl.nb; ++j) {
+          const int blk = __shfl_sync(0xffffffffu, my_blk, j);
+          if (lane == 0)
+            tma_load(s_base + kS_K + stage * kKStageBytes + j * kSlabBytes, &tm_kv,
+                     bar(kKFull + stage), 64 * k, blk * kRows);
+        }
+        __syncwarp();
       }
     }
-    if (ok && have_prev) issue_pv(t - 1);
-  } else {
-    // ------------------------------------------------------------------ softmax + epilogue
+    for (int k = 1; k <= kKStages && k <= kt; ++k)
+      drain_wait(bar(kKFull + (kt - k) % kKStages), ((kt - k) / kKStages) & 1, p.err);
+    if (seg_i > 0) drain_wait(bar(kQFull), (seg_i - 1) & 1, p.err);
+  } else if (score && warp == 1) {
+    // ---------------------------------------------------------------- score: S = Q . K^T
+    int kt = 0, t = 0, seg_i = 0;
+    bool ok = true;
+    while (ok && walk.next(tl)) {
+      if (tl.first) {
+        ok = warp_wait(bar(kQFull), seg_i & 1, ctl);
+        ++seg_i;
+      }
+      if (ok && t > 0) ok = warp_wait(bar(kSFree), (t - 1) & 1, ctl);
+      if (!ok) break;
+      const uint32_t id = idesc(128, kRows * tl.nb, 0);
+      for (int k = 0; k < 9; ++k, ++kt) {
+        const int stage = kt % kKStages;
+        if (!warp_wait(bar(kKFull + stage), (kt / kKStages) & 1, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_after();
+        if (lane == 0) {
+          const uint32_t kb = s_base + kS_K + stage * kKStageBytes;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {  // 16 dims per step; B K-major, 8-row groups 1024 B apart
+            const uint64_t bd = sdesc(kb + 32 * i, 16, 1024, 2);
+            const uint32_t acc = (k > 0 || i > 0) ? 1u : 0u;
+            if (k < 8)
+              mma_ts(tmem, tmem + 256 + 32 * k + 8 * i, bd, id, acc);
+            else
+              mma_ss(tmem, sdesc(s_base + kS_QRope + 32 * i, 16, 1024, 2), bd, id, acc);
+          }
+          tc_commit(bar(kKEmpty + stage));
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        tc_commit(bar(kSFull));
+        if (tl.last) tc_commit(bar(kQEmpty));
+      }
+      __syncwarp();
+      ++t;
+    }
+  } else if (score) {
+    // ---------------------------------------------------------------- score: softmax, P out
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
     const float c2 = p.scale * 1.4426950408889634f;  // scores in log2 units
     const __nv_bfloat16* Q = (const __nv_bfloat16*)p.q;
-    const uint32_t row_off = (uint32_t)h * (kRows * 4);
-    const uint32_t peer_inbox = peer_addr(s_inbox, peer);
-    uint32_t peer_xfull[kInboxSlots];
-#pragma unroll
-    for (int i = 0; i < kInboxSlots; ++i) peer_xfull[i] = peer_addr(bar(kXFull + i), peer);
-    const int swz = h & 15;
+    const uint32_t peer_slots = peer_addr(s_base + kV_P, peer);
+    const uint32_t peer_hdr = peer_addr(s_base + kV_Hdr, peer);
+    const uint32_t stage_p = s_base + kS_Stage;
+    const uint32_t hdr = s_base + kS_Hdr;
 
-    auto load_q = [&](int bt) {
+    auto load_qckv = [&](int bt) {  // latent part of Q into TMEM columns [256, 512)
       const uint4* src = (const uint4*)(Q + ((size_t)bt * kH + h) * kD);
-      uint32_t w[32];
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+#pragma unroll 1
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t w[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint4 v = src[(256 * rank + 64 * ch) / 8 + i];
+          const uint4 v = src[8 * ch + i];
           w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
         }
-        tmem_st32(tl + kColQ + 32 * ch, w);
+        tmem_st32(tq + 256 + 32 * ch, w);
       }
-      uint32_t wr[16];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = src[(kR + 32 * rank) / 8 + i];
-        wr[4 * i] = v.x; wr[4 * i + 1] = v.y; wr[4 * i + 2] = v.z; wr[4 * i + 3] = v.w;
-      }
-      tmem_st16(tl + kColQ + 128, wr);
       tmem_wait_st();
       tc_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kQFull));
     };
 
-    int t = 0;
+    int t = 0, g = 0;
     float m_ref = 0.f, l = 0.f;
-    bool ok = true;
-    if (sb < se) load_q(p.segments[sb].bt);
-    for (int s = sb; ok && s < se; ++s) {
-      const Segment sg = p.segments[s];
-      const int chunk0 = p.bt_chunk0[sg.bt];
-      const int len = p.bt_len[sg.bt];
-      for (int c = sg.chunk_lo; ok && c < sg.chunk_hi; ++c) {
-        const bool first = (c == sg.chunk_lo), last = (c == sg.chunk_hi - 1);
-        const int valid = min(kRows, len - (c - chunk0) * kRows);
-
-        // own partial scores
-        if (!warp_wait(bar(kSFull), t & 1, ctl)) { ok = false; break; }
-        tc_after();
-        uint32_t sv[64];
-        tmem_ld64(tl + kColS, sv);
-        tc_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kSFree));
-
-        // swap partials with the other CTA: write into its inbox slot, read ours
-        const int slot = t & 1;
-        const uint32_t pdst = peer_inbox + (uint32_t)slot * kInboxBytes + row_off;
+    bool ok = true, q_loaded = false;
+    while (ok && walk.next(tl)) {
+      if (!q_loaded) {
+        load_qckv(tl.bt);
+        q_loaded = true;
+      }
+      if (!warp_wait(bar(kSFull), t & 1, ctl)) break;
+      tc_after();
+      // pass 1: row max over the tile's valid rows
+      float mt = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < tl.nb; ++c) {
+        uint32_t v[64];
+        tmem_ld64(tq + 64 * c, v);
+        const int lim = tl.ntok - 64 * c;
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          st_async_peer(pdst + 16u * (uint32_t)(u ^ swz), sv[4 * u], sv[4 * u + 1], sv[4 * u + 2],
-                        sv[4 * u + 3], peer_xfull[slot]);
-        if (!warp_wait(bar(kXFull + slot), (t >> 1) & 1, ctl)) { ok = false; break; }
-        float x[64];
-        const uint32_t mine = s_inbox + (uint32_t)slot * kInboxBytes + row_off;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          uint4 v;
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                       : "r"(mine + 16u * (uint32_t)(u ^ swz))
-                       : "memory");
-          x[4 * u] = __uint_as_float(sv[4 * u]) + __uint_as_float(v.x);
-          x[4 * u + 1] = __uint_as_float(sv[4 * u + 1]) + __uint_as_float(v.y);
-          x[4 * u + 2] = __uint_as_float(sv[4 * u + 2]) + __uint_as_float(v.z);
-          x[4 * u + 3] = __uint_as_float(sv[4 * u + 3]) + __uint_as_float(v.w);
-        }
-        // this slot's next use is tile t + 2; the peer can only write it after receiving our
-        // partial of tile t + 1, so re-arming now cannot race with this tile's reads
-        if (threadIdx.x == 64) mbar_expect_tx(bar(kXFull + slot), kInboxBytes);
-
-        // online softmax in log2 units, lazy rescale of O
-        float mt = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          x[k] = (k < valid) ? x[k] * c2 : -INFINITY;
-          mt = fmaxf(mt, x[k]);
-        }
-        float alpha = 1.f;
-        bool rescale = false;
-        if (first) {
-          m_ref = mt;
-          l = 0.f;
-        } else if (mt > m_ref + 8.f) {
-          alpha = ex2(m_ref - mt);
-          m_ref = mt;
-          rescale = true;
-        }
-        float rs = 0.f;
+        for (int k = 0; k < 64; ++k)
+          if (k < lim) mt = fmaxf(mt, __uint_as_float(v[k]));
+      }
+      mt *= c2;
+      float alpha = 1.f;
+      if (tl.first) {
+        m_ref = mt;
+        l = 0.f;
+      } else if (mt > m_ref + 8.f) {
+        alpha = ex2(m_ref - mt);
+        m_ref = mt;
+      }
+      // the value CTA must have received the previous tile before staging is overwritten
+      if (t > 0 && !warp_wait(bar(kStgFree), (t - 1) & 1, ctl)) break;
+      // pass 2: P = exp2(s * c2 - m_ref), rounded to bf16, into the A-operand layout
+      float rs = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < tl.nb; ++c) {
+        uint32_t v[64];
+        tmem_ld64(tq + 64 * c, v);
+        const int lim = tl.ntok - 64 * c;
         uint32_t pw[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          const float p0 = ex2(x[2 * k] - m_ref);
-          const float p1 = ex2(x[2 * k + 1] - m_ref);
+          const float p0 = (2 * k < lim) ? ex2(__uint_as_float(v[2 * k]) * c2 - m_ref) : 0.f;
+          const float p1 = (2 * k + 1 < lim) ? ex2(__uint_as_float(v[2 * k + 1]) * c2 - m_ref) : 0.f;
           rs += p0;
           rs += p1;
           pw[k] = pack_bf16(p0, p1);
         }
-        l = l * alpha + rs;
-
-        // P . V of the previous tile must be done before P and O are touched
-        if (t > 0 && !warp_wait(bar(kPvDone), (t - 1) & 1, ctl)) { ok = false; break; }
-        tc_after();
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-          for (int ch = 0; ch < 8; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(tl + kColO + 32 * ch, o);
+        const uint32_t row = stage_p + c * kPBlockBytes + (uint32_t)h * 128;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tl + kColO + 32 * ch, o);
+        for (int u = 0; u < 8; ++u)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           row + 16u * (uint32_t)(u ^ (h & 7))),
+                       "r"(pw[4 * u]), "r"(pw[4 * u + 1]), "r"(pw[4 * u + 2]), "r"(pw[4 * u + 3])
+                       : "memory");
+      }
+      l = l * alpha + rs;
+      tc_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kSFree));  // S may be overwritten by the next tile
+      asm volatile("st.shared.f32 [%0], %1;" ::"r"(hdr + 4u * h), "f"(alpha) : "memory");
+      if (tl.last) asm volatile("st.shared.f32 [%0], %1;" ::"r"(hdr + 4u * (kH + h)), "f"(l) : "memory");
+      fence_proxy_async();
+      sync_math_warps();
+      if (warp == 2) {  // ship header and P blocks to the value CTA
+        bool slots_ok = true;
+        for (int c = 0; c < tl.nb && slots_ok; ++c) {
+          const int gb = g + c;
+          if (gb >= kPSlots)
+            slots_ok = warp_wait(bar(kSlotFree + gb % kPSlots), ((gb / kPSlots) - 1) & 1, ctl);
+        }
+        if (slots_ok && lane == 0) {
+          const int hs = t % kHdrSlots;
+          bulk_to_peer(peer_hdr + hs * kHdrBytes, hdr, kHdrBytes,
+                       peer_addr(bar(kHFull + hs), peer));
+          for (int c = 0; c < tl.nb; ++c) {
+            const int slot = (g + c) % kPSlots;
+            bulk_to_peer(peer_slots + slot * kPBlockBytes, stage_p + c * kPBlockBytes,
+                         kPBlockBytes, peer_addr(bar(kPFull + slot), peer));
           }
         }
-        tmem_st32(tl + kColP, pw);
-        tmem_wait_st();
-        tc_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kPFull));
-        ++t;
-
-        if (last) {
-          // next segment's query goes in while this segment drains
-          if (s + 1 < se) load_q(p.segments[s + 1].bt);
-          if (!warp_wait(bar(kPvDone), (t - 1) & 1, ctl)) { ok = false; break; }
-          tc_after();
-          const float inv_l = 1.f / l;
-          const float lse = (m_ref + __log2f(l)) * 0.6931471805599453f;
-          float* dst = (sg.slot < 0 ? p.out + ((size_t)sg.bt * kH + h) * kR
-                                    : p.part_o + ((size_t)sg.slot * kH + h) * kR) +
-                       256 * rank;
-#pragma unroll 1
-          for (int ch = 0; ch < 8; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(tl + kColO + 32 * ch, o);
-            float4* d4 = (float4*)(dst + 32 * ch);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              d4[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l,
-                                  __uint_as_float(o[4 * i + 1]) * inv_l,
-                                  __uint_as_float(o[4 * i + 2]) * inv_l,
-                                  __uint_as_float(o[4 * i + 3]) * inv_l);
+        if (!slots_ok) ok = false;
+      }
+      if (tl.last) {
+        const float lse = (m_ref + __log2f(l)) * 0.6931471805599453f;
+        if (tl.slot < 0) {
+          if (p.lse) p.lse[(size_t)tl.bt * kH + h] = lse;
+        } else {
+          p.part_lse[(size_t)tl.slot * kH + h] = lse;
+        }
+        // the next segment's query: this segment's last S product is complete
+        TileWalk look = walk;
+        Tile nx;
+        if (look.next(nx)) load_qckv(nx.bt);
+      }
+      g += tl.nb;
+      ++t;
+    }
+  } else if (warp == 0) {
+    // ---------------------------------------------------------------- value: TMA producer
+    int vt = 0;
+    bool ok = true;
+    while (ok && walk.next(tl)) {
+      const int my_blk = tile_block(p, tl, lane);
+      for (int j = 0; j < tl.nb && ok; ++j) {
+        const int blk = __shfl_sync(0xffffffffu, my_blk, j);
+        for (int dh = 0; dh < 2; ++dh, ++vt) {
+          const int vs = vt % kVStages;
+          if (vt >= kVStages && !warp_wait(bar(kVEmpty + vs), ((vt / kVStages) - 1) & 1, ctl)) {
+            ok = false;
+            break;
           }
-          if (rank == 0) {
-            if (sg.slot < 0) {
-              if (p.lse) p.lse[(size_t)sg.bt * kH + h] = lse;
-            } else {
-              p.part_lse[(size_t)sg.slot * kH + h] = lse;
-            }
+          if (lane == 0) {
+            mbar_expect_tx(bar(kVFull + vs), kVStageBytes);
+            for (int i = 0; i < 4; ++i)
+              tma_load(s_base + kV_V + vs * kVStageBytes + i * kSlabBytes, &tm_kv,
+                       bar(kVFull + vs), 256 * dh + 64 * i, blk * kRows);
           }
-          tc_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kOFree));
         }
       }
+    }
+    for (int k = 1; k <= kVStages && k <= vt; ++k)
+      drain_wait(bar(kVFull + (vt - k) % kVStages), ((vt - k) / kVStages) & 1, p.err);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- value: O += P . V
+    int vt = 0, g = 0, t = 0;
+    bool ok = true;
+    while (ok && walk.next(tl)) {
+      // the whole tile's P and header arrived: the score CTA may reuse its staging
+      for (int j = 0; j < tl.nb && ok; ++j)
+        ok = warp_wait(bar(kPFull + (g + j) % kPSlots), ((g + j) / kPSlots) & 1, ctl);
+      if (ok) ok = warp_wait(bar(kHFull + t % kHdrSlots), (t / kHdrSlots) & 1, ctl);
+      if (ok) ok = warp_wait(bar(kOReady), t & 1, ctl);
+      if (!ok) break;
+      if (lane == 0) {
+        for (int j = 0; j < tl.nb; ++j)  // re-arm for each slot's next use
+          mbar_expect_tx(bar(kPFull + (g + j) % kPSlots), kPBlockBytes);
+        mbar_arrive_peer(peer_addr(bar(kStgFree), peer));
+      }
+      __syncwarp();
+      for (int j = 0; j < tl.nb && ok; ++j, ++g) {
+        const int slot = g % kPSlots;
+        const int valid = min(kRows, tl.ntok - kRows * j);
+        for (int dh = 0; dh < 2; ++dh, ++vt) {
+          const int vs = vt % kVStages;
+          if (!warp_wait(bar(kVFull + vs), (vt / kVStages) & 1, ctl)) {
+            ok = false;
+            break;
+          }
+          if (valid < kRows) {
+            // rows past the sequence end: zero them so 0 * garbage never enters P . V
+            uint8_t* st = smem + kV_V + vs * kVStageBytes;
+            const int n16 = (kRows - valid) * 128 / 16;
+            for (int slab = 0; slab < 4; ++slab) {
+              uint4* z = (uint4*)(st + slab * kSlabBytes + valid * 128);
+              for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async();
+            __syncwarp();
+          }
+          tc_after();
+          if (lane == 0) {
+            const uint32_t vb = s_base + kV_V + vs * kVStageBytes;
+            const uint32_t pb = s_base + kV_P + slot * kPBlockBytes;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)  // 16 rows per step; B MN-major: LBO = 64-dim slab
+              mma_ss(tmem + 256 * dh, sdesc(pb + 32 * i, 16, 1024, 2),
+                     sdesc(vb + 2048 * i, kSlabBytes, 1024, 2), kIdescPV,
+                     (tl.first && j == 0 && i == 0) ? 0u : 1u);
+            tc_commit(bar(kVEmpty + vs));
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (lane == 0) tc_commit(bar(kSlotDone + slot));
+        __syncwarp();
+        if (g >= 2) {  // slot of block g - 2 is free once its P . V completed
+          const int gb = g - 2;
+          if (!warp_wait(bar(kSlotDone + gb % kPSlots), (gb / kPSlots) & 1, ctl)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive_peer(peer_addr(bar(kSlotFree + gb % kPSlots), peer));
+          __syncwarp();
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(bar(kPvDone + (t & 1)));
+      __syncwarp();
+      ++t;
+    }
+  } else {
+    // ---------------------------------------------------------------- value: rescale, epilogue
+    const int quad = warp & 3;
+    const int h = quad * 32 + lane;
+    const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
+    int t = 0;
+    float l_last = 1.f;
+    bool ok = true;
+    // Completions of P . V are observed tile by tile, in order: a parity wait is only
+    // unambiguous when the phase before it has been seen. Tile k's phase on barrier k & 1 can
+    // only be followed by tile k + 2's, which needs this warp's OReady of tile k + 2 first.
+    int pv_next = 0;
+    auto wait_pv = [&](int k) -> bool {
+      while (pv_next <= k) {
+        if (!warp_wait(bar(kPvDone + (pv_next & 1)), (pv_next >> 1) & 1, ctl)) return false;
+        ++pv_next;
+      }
+      return true;
+    };
+    while (ok && walk.next(tl)) {
+      const int hs = t % kHdrSlots;
+      if (!warp_wait(bar(kHFull + hs), (t / kHdrSlots) & 1, ctl)) break;
+      const uint32_t hb = s_base + kV_Hdr + hs * kHdrBytes;
+      float alpha;
+      asm volatile("ld.shared.f32 %0, [%1];" : "=f"(alpha) : "r"(hb + 4u * h) : "memory");
+      if (tl.last) asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l_last) : "r"(hb + 4u * (kH + h)) : "memory");
+      sync_math_warps();  // everyone has read the header before it is re-armed
+      if (threadIdx.x == 64) mbar_expect_tx(bar(kHFull + hs), kHdrBytes);
+      if (!tl.first && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!wait_pv(t - 1)) break;
+        tc_after();
+#pragma unroll 1
+        for (int ch = 0; ch < 16; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(tq + 32 * ch, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tq + 32 * ch, o);
+        }
+        tmem_wait_st();
+      }
+      tc_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kOReady));
+      if (!tl.last) {
+        if (t > 0 && !wait_pv(t - 1)) break;  // keep up with completions
+      } else {
+        if (!wait_pv(t)) break;
+        tc_after();
+        const float inv_l = 1.f / l_last;
+        float* dst = tl.slot < 0 ? p.out + ((size_t)tl.bt * kH + h) * kR
+                                 : p.part_o + ((size_t)tl.slot * kH + h) * kR;
+#pragma unroll 1
+        for (int ch = 0; ch < 16; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(tq + 32 * ch, o);
+          float4* d4 = (float4*)(dst + 32 * ch);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            d4[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l,
+                                __uint_as_float(o[4 * i + 1]) * inv_l,
+                                __uint_as_float(o[4 * i + 2]) * inv_l,
+                                __uint_as_float(o[4 * i + 3]) * inv_l);
+        }
+        tc_before();
+      }
+      ++t;
     }
   }
 
@@ -601,11 +787,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_ckv,
   if (warp == 1) {
     if (lane == 0) tc_commit(bar(kFinal));  // completes once every MMA issued here is done
     __syncwarp();
-    const uint64_t t0 = globaltimer();
-    bool done = false;
-    while (!done && globaltimer() - t0 < kTimeoutNs)
-      done = __all_sync(0xffffffffu, mbar_try(bar(kFinal), 0));
-    if (!done && lane == 0) set_error(p.err, MLA_DEV_WAIT_TIMEOUT);
+    drain_wait(bar(kFinal), 0, p.err);
     __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
@@ -629,17 +811,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-bool make_map(CUtensorMap* m, const void* pool, int num_blocks, uint32_t box_cols,
-              CUtensorMapSwizzle swz) {
+// 2-D bf16 view [rows][576] with 128-byte swizzled boxes of 64 columns x box_rows rows.
+bool make_map(CUtensorMap* m, const void* base, long long rows, uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)num_blocks * kRows};
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-  cuuint32_t box[2] = {box_cols, (cuuint32_t)kRows};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -651,9 +833,9 @@ bool tc_supported(const mla_config& c) {
 
 cudaError_t launch_attend_tc(const mla_config& c, const DecodeParams& p, cudaStream_t st) {
   (void)c;
-  CUtensorMap ckv, rope;
-  if (!make_map(&ckv, p.pool, p.num_blocks, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&rope, p.pool, p.num_blocks, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+  CUtensorMap kv, qm;
+  if (!make_map(&kv, p.pool, (long long)p.num_blocks * kRows, kRows) ||
+      !make_map(&qm, p.q, (long long)p.BT * kH, kH))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
@@ -662,7 +844,7 @@ cudaError_t launch_attend_tc(const mla_config& c, const DecodeParams& p, cudaStr
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  attend_tc_kernel<<<2 * kRanges, kThreads, kSmemBytes, st>>>(ckv, rope, p);
+  attend_tc_kernel<<<2 * kRanges, kThreads, kSmemBytes, st>>>(kv, qm, p);
   return cudaGetLastError();
 }
 
