@@ -21,7 +21,9 @@
 //   * the value CTA streams the latent part of the same rows by TMA and accumulates O = P . V
 //     in its whole TMEM, applies rescales, and writes the normalised output.
 // The two read the same cache blocks close together in time, so HBM sees each row about once.
-// Warps: 0 TMA, 1 MMA issue, 2-5 softmax (score CTA) or rescale and epilogue (value CTA).
+// Warps: 0 TMA, 1 MMA issue, 2-5 softmax (score CTA) or rescale and epilogue (value CTA), 6
+// the cross-CTA traffic (bulk copies out of the score CTA, acknowledgements out of the value
+// CTA), so that no MMA-issuing warp ever waits on a cluster-scope fence.
 // Every wait is bounded: on timeout the kernel sets MLA_DEV_WAIT_TIMEOUT, drains its copies
 // and MMAs, frees TMEM and returns. No TMA multicast is used.
 #include <cuda.h>
@@ -39,7 +41,7 @@ constexpr int kD = kR + kDR;
 constexpr int kRows = 64;                       // rows per cache block = planner chunk
 constexpr int kTileBlocks = 4;                  // blocks per score tile (N <= 256)
 constexpr int kSlabBytes = kRows * 64 * 2;      // 64 rows x 64 dims bf16: 8 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;  // 7 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kTimeoutNs = 1000000000ull;  // 1 s per wait
 
@@ -74,6 +76,7 @@ enum Bar {
   kSFull,                       // S complete
   kSFree,                       // softmax done reading S
   kStgFree,                     // value CTA received the previous tile's P (staging reusable)
+  kStaged,                      // softmax warps finished writing a tile's P and header
   kSlotFree,                    // kPSlots: value CTA finished with a P ring slot
   // value CTA
   kVFull = kSlotFree + kPSlots,
@@ -368,6 +371,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       mbar_init(bar(kSFull), 1);
       mbar_init(bar(kSFree), 4);
       mbar_init(bar(kStgFree), 1);
+      mbar_init(bar(kStaged), 4);
       for (int i = 0; i < kPSlots; ++i) mbar_init(bar(kSlotFree + i), 1);
     } else {
       for (int i = 0; i < kVStages; ++i) {
@@ -488,15 +492,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       __syncwarp();
       ++t;
     }
-  } else if (score) {
-    // ---------------------------------------------------------------- score: softmax, P out
+  } else if (score && warp < 6) {
+    // ---------------------------------------------------------------- score: softmax, P staged
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
     const float c2 = p.scale * 1.4426950408889634f;  // scores in log2 units
     const __nv_bfloat16* Q = (const __nv_bfloat16*)p.q;
-    const uint32_t peer_slots = peer_addr(s_base + kV_P, peer);
-    const uint32_t peer_hdr = peer_addr(s_base + kV_Hdr, peer);
     const uint32_t stage_p = s_base + kS_Stage;
     const uint32_t hdr = s_base + kS_Hdr;
 
@@ -580,27 +582,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       if (lane == 0) mbar_arrive(bar(kSFree));  // S may be overwritten by the next tile
       asm volatile("st.shared.f32 [%0], %1;" ::"r"(hdr + 4u * h), "f"(alpha) : "memory");
       if (tl.last) asm volatile("st.shared.f32 [%0], %1;" ::"r"(hdr + 4u * (kH + h)), "f"(l) : "memory");
-      fence_proxy_async();
-      sync_math_warps();
-      if (warp == 2) {  // ship header and P blocks to the value CTA
-        bool slots_ok = true;
-        for (int c = 0; c < tl.nb && slots_ok; ++c) {
-          const int gb = g + c;
-          if (gb >= kPSlots)
-            slots_ok = warp_wait(bar(kSlotFree + gb % kPSlots), ((gb / kPSlots) - 1) & 1, ctl);
-        }
-        if (slots_ok && lane == 0) {
-          const int hs = t % kHdrSlots;
-          bulk_to_peer(peer_hdr + hs * kHdrBytes, hdr, kHdrBytes,
-                       peer_addr(bar(kHFull + hs), peer));
-          for (int c = 0; c < tl.nb; ++c) {
-            const int slot = (g + c) % kPSlots;
-            bulk_to_peer(peer_slots + slot * kPBlockBytes, stage_p + c * kPBlockBytes,
-                         kPBlockBytes, peer_addr(bar(kPFull + slot), peer));
-          }
-        }
-        if (!slots_ok) ok = false;
-      }
+      fence_proxy_async();  // staged bytes are read by the bulk copies (async proxy)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kStaged));
       if (tl.last) {
         const float lse = (m_ref + __log2f(l)) * 0.6931471805599453f;
         if (tl.slot < 0) {
@@ -614,6 +598,54 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
         if (look.next(nx)) load_qckv(nx.bt);
       }
       g += tl.nb;
+      ++t;
+    }
+  } else if (score && warp == 6) {
+    // ---------------------------------------------------------------- score: ship P out
+    const uint32_t peer_slots = peer_addr(s_base + kV_P, peer);
+    const uint32_t peer_hdr = peer_addr(s_base + kV_Hdr, peer);
+    int t = 0, g = 0;
+    bool ok = true;
+    while (ok && walk.next(tl)) {
+      ok = warp_wait(bar(kStaged), t & 1, ctl);
+      for (int c = 0; c < tl.nb && ok; ++c) {  // the ring slot's previous block is done
+        const int gb = g + c;
+        if (gb >= kPSlots)
+          ok = warp_wait(bar(kSlotFree + gb % kPSlots), ((gb / kPSlots) - 1) & 1, ctl);
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        const int hs = t % kHdrSlots;
+        bulk_to_peer(peer_hdr + hs * kHdrBytes, s_base + kS_Hdr, kHdrBytes,
+                     peer_addr(bar(kHFull + hs), peer));
+        for (int c = 0; c < tl.nb; ++c) {
+          const int slot = (g + c) % kPSlots;
+          bulk_to_peer(peer_slots + slot * kPBlockBytes, s_base + kS_Stage + c * kPBlockBytes,
+                       kPBlockBytes, peer_addr(bar(kPFull + slot), peer));
+        }
+      }
+      __syncwarp();
+      g += tl.nb;
+      ++t;
+    }
+  } else if (!score && warp == 6) {
+    // ---------------------------------------------------------------- value: acknowledgements
+    int t = 0, g = 0;
+    bool ok = true;
+    while (ok && walk.next(tl)) {
+      // the whole tile arrived: the score CTA may overwrite its staging
+      for (int j = 0; j < tl.nb && ok; ++j)
+        ok = warp_wait(bar(kPFull + (g + j) % kPSlots), ((g + j) / kPSlots) & 1, ctl);
+      if (ok) ok = warp_wait(bar(kHFull + t % kHdrSlots), (t / kHdrSlots) & 1, ctl);
+      if (!ok) break;
+      if (lane == 0) mbar_arrive_peer(peer_addr(bar(kStgFree), peer));
+      __syncwarp();
+      // each ring slot is free once the P . V that read it completed
+      for (int j = 0; j < tl.nb && ok; ++j, ++g) {
+        ok = warp_wait(bar(kSlotDone + g % kPSlots), (g / kPSlots) & 1, ctl);
+        if (ok && lane == 0) mbar_arrive_peer(peer_addr(bar(kSlotFree + g % kPSlots), peer));
+        __syncwarp();
+      }
       ++t;
     }
   } else if (warp == 0) {
@@ -653,11 +685,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       if (ok) ok = warp_wait(bar(kHFull + t % kHdrSlots), (t / kHdrSlots) & 1, ctl);
       if (ok) ok = warp_wait(bar(kOReady), t & 1, ctl);
       if (!ok) break;
-      if (lane == 0) {
+      if (lane == 0)
         for (int j = 0; j < tl.nb; ++j)  // re-arm for each slot's next use
           mbar_expect_tx(bar(kPFull + (g + j) % kPSlots), kPBlockBytes);
-        mbar_arrive_peer(peer_addr(bar(kStgFree), peer));
-      }
       __syncwarp();
       for (int j = 0; j < tl.nb && ok; ++j, ++g) {
         const int slot = g % kPSlots;
@@ -695,15 +725,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
         if (!ok) break;
         if (lane == 0) tc_commit(bar(kSlotDone + slot));
         __syncwarp();
-        if (g >= 2) {  // slot of block g - 2 is free once its P . V completed
-          const int gb = g - 2;
-          if (!warp_wait(bar(kSlotDone + gb % kPSlots), (gb / kPSlots) & 1, ctl)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) mbar_arrive_peer(peer_addr(bar(kSlotFree + gb % kPSlots), peer));
-          __syncwarp();
-        }
       }
       if (!ok) break;
       if (lane == 0) tc_commit(bar(kPvDone + (t & 1)));
