@@ -47,6 +47,27 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def max_over_ranks(values, world: int, device="cpu"):
+    """Element-wise max of a list of floats over all ranks (the slowest rank's times)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def aggregate_rate(units_per_rank_step: float, world: int, steps: int, elapsed_ms: float):
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return units_per_rank_step * world * steps / (elapsed_ms * 1e-3)
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's own batch: every replica decodes different sequences."""
+    return rank
+
+
 def workload_desc(w):
     return (f"{w.name}: H={w.num_heads} d_h={w.head_dim} r={w.kv_rank} d_r={w.rope_dim} "
             f"B={w.batch} S={w.cached if not w.ragged_max else 'U[1,%d]' % w.ragged_max} "
@@ -63,65 +84,107 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------------------
-# clocks sampled by nvidia-smi while the timed region runs
+# SM clocks and clock-event reasons, read through NVML every 10 ms by a host thread while the
+# timed region runs (read-only queries; nothing is set). nvidia-smi is the fallback.
 # ---------------------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id: str):
-        self.samples = []
-        self.proc = None
-        self.gpu_id = gpu_id
-        self.window = None
+    def __init__(self, uuid: str, index: int, period_s: float = 0.01):
+        self.uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        self.index = index
+        self.period = period_s
+        self.samples = []          # (time, sm_mhz, max_mhz, [reasons])
+        self.source = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            except pynvml.NVMLError:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            masks = [(n, getattr(pynvml, a)) for n, a in self.REASONS if hasattr(pynvml, a)]
+            self.source = "nvml"
+            self._thread = threading.Thread(target=self._nvml_loop, args=(pynvml, h, masks),
+                                            daemon=True)
+            self._thread.start()
+        except Exception:  # no NVML binding or library: nvidia-smi at its fastest period
+            self._start_smi()
+        t_end = time.time() + 5.0
+        while not self.samples and time.time() < t_end:
+            time.sleep(0.01)
+
+    def _nvml_loop(self, pynvml, h, masks):
+        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.time(), float(sm), float(mx),
+                                     [n for n, m in masks if bits & m]))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def _start_smi(self):
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.SMI_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
-            self.proc = None
             return
-        threading.Thread(target=self._read, daemon=True).start()
+        self.source = "nvidia-smi"
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.samples.append((time.time(), line.strip()))
+        def read():
+            for line in self._proc.stdout:
+                parts = [p.strip() for p in line.split(",")]
+                try:
+                    self.samples.append((time.time(), float(parts[0]), float(parts[1]),
+                                         [n for n, v in zip(names, parts[4:8])
+                                          if v.lower() == "active"]))
+                except (ValueError, IndexError):
+                    continue
+        threading.Thread(target=read, daemon=True).start()
 
     def stop(self):
-        if self.proc:
-            self.proc.terminate()
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=2)
+        if self._proc:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
+                self._proc.kill()
 
     def summary(self, t0, t1):
-        rows = [(t, s) for t, s in self.samples if t0 <= t <= t1]
+        rows = [s for s in self.samples if t0 <= s[0] <= t1]
         window = "timed region"
         if not rows and self.samples:
             mid = 0.5 * (t0 + t1)
-            rows = sorted(self.samples, key=lambda x: abs(x[0] - mid))[:3]
-            window = "nearest samples to a timed region shorter than the sampling period"
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for _, s in rows:
-            parts = [p.strip() for p in s.split(",")]
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except (ValueError, IndexError):
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm), "window": window}
+            rows = sorted(self.samples, key=lambda s: abs(s[0] - mid))[:3]
+            window = "nearest samples to the timed region"
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": self.source}
+        reasons = sorted({n for s in rows for n in s[3]})
+        return {"sm_mhz": statistics.median(s[1] for s in rows),
+                "sm_max_mhz": max(s[2] for s in rows), "reasons": reasons,
+                "samples": len(rows), "window": window, "source": self.source}
 
 
 # ---------------------------------------------------------------------------------------
@@ -231,7 +294,7 @@ def run_ours(args, w):
                                 device_id=dev)
     kernel = {"auto": mla.DECODE_AUTO, "simt": mla.DECODE_SIMT,
               "tensor": mla.DECODE_TENSOR}[args.decode_kernel]
-    st = DecodeState(w, seed=rank, device=str(dev), decode_kernel=kernel)
+    st = DecodeState(w, seed=rank_seed(rank), device=str(dev), decode_kernel=kernel)
     stream = torch.cuda.Stream(device=dev)
     B, T = w.batch, w.new_tokens
     tokens_per_step = B * T
@@ -252,11 +315,10 @@ def run_ours(args, w):
     names = ["absorb", "append", "plan", "attend", "combine", "output"]
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
           for _ in range(args.steps)]
-    clock = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid)
-                         if hasattr(torch.cuda.get_device_properties(dev), "uuid") else str(local))
+    props = torch.cuda.get_device_properties(dev)
+    clock = ClockSampler(str(getattr(props, "uuid", "")), local)
     if rank == 0:
         clock.start()
-        time.sleep(0.3)
     barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
@@ -317,10 +379,8 @@ def run_ours(args, w):
     barrier()
 
     # ---- max over ranks ----
-    t = torch.tensor([elapsed_ms, e2e_ms, stage_ms["attend"]], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms, attend_ms = (float(x) for x in t.tolist())
+    elapsed_ms, e2e_ms, attend_ms = max_over_ranks([elapsed_ms, e2e_ms, stage_ms["attend"]],
+                                                   world, dev)
     if rank == 0:
         clock.stop()
     clocks = clock.summary(t_wall0, t_wall1) if rank == 0 else None
@@ -356,8 +416,8 @@ def run_ours(args, w):
                  "tensor_view": {"achieved_tflops": tflops, "peak": tc_burst,
                                  "frac": tflops / tc_burst}})
     ms_per_step = elapsed_ms / args.steps
-    value = tokens_per_step * world * args.steps / (elapsed_ms * 1e-3)
-    e2e_value = tokens_per_step * world * e2e_steps / (e2e_ms * 1e-3)
+    value = aggregate_rate(tokens_per_step, world, args.steps, elapsed_ms)
+    e2e_value = aggregate_rate(tokens_per_step, world, e2e_steps, e2e_ms)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,

@@ -36,7 +36,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 1
+#define MLA_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MLA_API __attribute__((visibility("default")))
@@ -54,8 +54,12 @@ typedef enum {
 
 typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
 
-/* Which attention kernel mla_decode uses. AUTO picks the tcgen05 tensor-core kernel for
- * bf16 at H=128, r=512, d_r=64, block_size=64, and the CUDA-core kernel otherwise. */
+/* Which kernels the calls use. AUTO: tcgen05 tensor-core kernels where dtype and shape allow
+ * them -- mla_decode's attention for bf16 at H=128, r=512, d_r=64, block_size=64; the
+ * projections of mla_absorb_query (d_h a multiple of 64 up to 256, r a multiple of 64) and
+ * mla_output (r a multiple of 64) for bf16 -- and CUDA-core kernels otherwise. SIMT: CUDA-core
+ * kernels for every call. TENSOR: tensor-core kernels, MLA_ERR_UNSUPPORTED where the shape
+ * has none. (The name is historical: the choice covers every call, not only mla_decode.) */
 typedef enum { MLA_DECODE_AUTO = 0, MLA_DECODE_SIMT = 1, MLA_DECODE_TENSOR = 2 } mla_decode_kernel;
 
 typedef struct {
@@ -89,10 +93,12 @@ typedef struct {
  * pos (n_tokens) int32 >= 0; w_uk (H, d_h, r) dtype -- the nn.Linear(r, H*d_h) weight,
  * rows h*d_h .. (h+1)*d_h-1 for head h, i.e. the same memory without a transpose;
  * q_out (n_tokens, H, r + d_r) dtype, rounded to nearest even when bf16.
+ * dev_err may be NULL; the tensor-core kernel sets MLA_DEV_WAIT_TIMEOUT in it when one of its
+ * bounded waits gives up (that tile of q_out is then not written).
  */
 MLA_API mla_status mla_absorb_query(const mla_config* cfg, const void* q_nope, const void* q_rope,
                             const int32_t* pos, const void* w_uk, void* q_out, int32_t n_tokens,
-                            void* stream);
+                            uint32_t* dev_err, void* stream);
 
 /*
  * mla_append_latent -- [B] (norm_kv before caching; paged cache), [C] (append), [D] (row
@@ -130,7 +136,8 @@ MLA_API size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, i
  * q (batch * q_per_seq, H, r + d_r) dtype; pool and block_table as in mla_append_latent;
  * seq_lens (batch) int32: rows valid after this step's append (callers advance it by
  * q_per_seq before the call); out_latent (batch * q_per_seq, H, r) float32;
- * lse (batch * q_per_seq, H) float32 or NULL. Runs three stages on `stream`: a one-CTA
+ * lse (batch * q_per_seq, H) float32 or NULL. q, pool and out_latent must be 16-byte aligned
+ * (MLA_ERR_INVALID_ARG otherwise). Runs three stages on `stream`: a one-CTA
  * planner that cuts all (sequence, token) row ranges into equal 64-row chunks of work, the
  * attention kernel, and a log-sum-exp combine of sequences that were split. A length outside
  * [1, max_blocks * block_size] sets MLA_DEV_BAD_LENGTH and that row's output is 0 (lse -inf).
@@ -187,9 +194,13 @@ MLA_API mla_status mla_decode_static_workspace(const mla_config* cfg, const void
  * output": o[n, h, :] = W_UV[h] out_latent[n, h, :] (fp32 accumulation).
  * out_latent (n_tokens, H, r) float32; w_uv (H, d_v, r) dtype (the nn.Linear(r, H*d_v)
  * weight); o (n_tokens, H, d_v) dtype. W_O is not part of the library.
+ * For bf16 the tensor-core kernel feeds out_latent to its bf16 MMA as two terms, hi = bf16(x)
+ * and lo = bf16(x - hi) (about 16 significant bits of x); the products are summed in fp32.
+ * The tensor-core kernel is used only when out_latent and w_uv are 16-byte aligned.
+ * dev_err may be NULL; it receives MLA_DEV_WAIT_TIMEOUT as for mla_absorb_query.
  */
 MLA_API mla_status mla_output(const mla_config* cfg, const float* out_latent, const void* w_uv, void* o,
-                      int32_t n_tokens, void* stream);
+                      int32_t n_tokens, uint32_t* dev_err, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 MLA_API const char* mla_status_string(mla_status status);

@@ -46,7 +46,7 @@ def _load():
     lib = ctypes.CDLL(LIB_PATH)
     P = ctypes.POINTER(MlaConfig)
     sig = {
-        "mla_absorb_query": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _c_i32, _vp]),
+        "mla_absorb_query": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _c_i32, _vp, _vp]),
         "mla_append_latent": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _vp,
                                        _c_i32, _c_i32, _vp, _vp]),
         "mla_decode_workspace_size": (_sz, [P, _c_i32, _c_i32]),
@@ -54,7 +54,7 @@ def _load():
                                 _vp, _vp, _vp, _vp]),
         "mla_decode_stages": (_c_i32, [P, _c_i32, _vp, _vp, _vp, _c_i32, _c_i32, _vp, _c_i32,
                                        _c_i32, _vp, _sz, _vp, _vp, _vp, _vp]),
-        "mla_output": (_c_i32, [P, _vp, _vp, _vp, _c_i32, _vp]),
+        "mla_output": (_c_i32, [P, _vp, _vp, _vp, _c_i32, _vp, _vp]),
         "mla_decode_static_workspace": (_c_i32, [P, _vp, _vp, _vp, _c_i32, _c_i32, _vp, _c_i32,
                                                  _c_i32, _vp, _vp, _vp, _vp]),
         "mla_status_string": (ctypes.c_char_p, [_c_i32]),
@@ -138,12 +138,12 @@ def _check(st: int, where: str):
         raise MlaError(st, where)
 
 
-def absorb_query(cfg: Config, q_nope, q_rope, pos, w_uk, q_out, stream=None):
+def absorb_query(cfg: Config, q_nope, q_rope, pos, w_uk, q_out, stream=None, dev_err=None):
     """mla_absorb_query: q_out[n, h] = [W_UK[h]^T q_nope[n, h] || RoPE(q_rope[n, h], pos[n])]."""
     c = cfg.c()
     _check(lib.mla_absorb_query(ctypes.byref(c), _ptr(q_nope), _ptr(q_rope), _ptr(pos),
-                                _ptr(w_uk), _ptr(q_out), int(q_nope.shape[0]), _stream(stream)),
-           "mla_absorb_query")
+                                _ptr(w_uk), _ptr(q_out), int(q_nope.shape[0]), _ptr(dev_err),
+                                _stream(stream)), "mla_absorb_query")
 
 
 def append_latent(cfg: Config, ckv_raw, krope_raw, gamma, seq_idx, pos, block_table, pool,
@@ -186,11 +186,11 @@ def decode_static_workspace(cfg: Config, q, pool, block_table, seq_lens, q_per_s
            "mla_decode_static_workspace")
 
 
-def output(cfg: Config, out_latent, w_uv, o, stream=None):
+def output(cfg: Config, out_latent, w_uv, o, stream=None, dev_err=None):
     """mla_output: o[n, h] = W_UV[h] out_latent[n, h]."""
     c = cfg.c()
     _check(lib.mla_output(ctypes.byref(c), _ptr(out_latent), _ptr(w_uv), _ptr(o),
-                          int(out_latent.shape[0]), _stream(stream)), "mla_output")
+                          int(out_latent.shape[0]), _ptr(dev_err), _stream(stream)), "mla_output")
 
 
 def abi_version() -> int:

@@ -129,5 +129,12 @@ bool tc_supported(const mla_config& c);
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_output(const mla_config& c, const float* lat, const void* w_uv, void* o,
                           int n, cudaStream_t st);
+bool absorb_tc_supported(const mla_config& c);
+bool output_tc_supported(const mla_config& c);
+cudaError_t launch_absorb_tc(const mla_config& c, const void* q_nope, const void* q_rope,
+                             const int32_t* pos, const void* w_uk, void* q_out, int n,
+                             uint32_t* err, cudaStream_t st);
+cudaError_t launch_output_tc(const mla_config& c, const float* lat, const void* w_uv, void* o,
+                             int n, uint32_t* err, cudaStream_t st);
 
 }  // namespace mla

@@ -24,26 +24,47 @@ __device__ __forceinline__ int range_start(int64_t q, int64_t R, int64_t C) {
 
 constexpr int kPlanThreads = 1024;
 
-// Inclusive block scan of two ints over kPlanThreads threads.
+// Inclusive block scan of two ints over kPlanThreads threads: shuffle scans inside each warp,
+// then one warp scans the 32 warp totals. s_a / s_b hold at least 32 ints.
 __device__ void block_scan2(int* s_a, int* s_b, int& a, int& b) {
-  const int tid = threadIdx.x;
-  s_a[tid] = a;
-  s_b[tid] = b;
-  __syncthreads();
-  for (int off = 1; off < kPlanThreads; off <<= 1) {
-    const int va = tid >= off ? s_a[tid - off] : 0;
-    const int vb = tid >= off ? s_b[tid - off] : 0;
-    __syncthreads();
-    s_a[tid] += va;
-    s_b[tid] += vb;
-    __syncthreads();
+  static_assert(kPlanThreads == 32 * 32, "one warp scans the warp totals");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int va = __shfl_up_sync(0xffffffffu, a, o), vb = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) {
+      a += va;
+      b += vb;
+    }
   }
-  a = s_a[tid];
-  b = s_b[tid];
+  if (lane == 31) {
+    s_a[warp] = a;
+    s_b[warp] = b;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int wa = s_a[lane], wb = s_b[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int va = __shfl_up_sync(0xffffffffu, wa, o), vb = __shfl_up_sync(0xffffffffu, wb, o);
+      if (lane >= o) {
+        wa += va;
+        wb += vb;
+      }
+    }
+    s_a[lane] = wa;
+    s_b[lane] = wb;
+  }
+  __syncthreads();
+  if (warp > 0) {
+    a += s_a[warp - 1];
+    b += s_b[warp - 1];
+  }
+  __syncthreads();  // s_a / s_b are reused by the next scan
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p) {
-  __shared__ int s_a[kPlanThreads], s_b[kPlanThreads];
+  __shared__ int s_a[32], s_b[32];
   __shared__ int s_carry_a, s_carry_b;
   const int tid = threadIdx.x;
   const int64_t cap = (int64_t)p.max_blocks * p.bs;
@@ -135,48 +156,56 @@ cudaError_t launch_plan(const DecodeParams& p, cudaStream_t st) {
 
 // ------------------------------------------------------------------------------------------
 // Combine: out = sum_i exp(lse_i - L) * o_i, L = log sum_i exp(lse_i), in segment order.
-// One CTA per (row group, 4 heads); row groups with a single segment were written directly by
-// the attention kernel and are skipped; row groups with an invalid length get 0 and -inf.
+// One CTA per (row group, 4 heads), one warp per head. Row groups with a single segment were
+// written directly by the attention kernel and are skipped; row groups with an invalid length
+// get 0 and -inf. The weights exp(lse_i - L) are computed once per (row group, head) into
+// shared memory; the partial rows are then streamed as float4 (a lane holds 4 of the r dims).
 // ------------------------------------------------------------------------------------------
 constexpr int kCombineHeads = 4;
 
-__global__ void __launch_bounds__(128) combine_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kCombineHeads * 32) combine_kernel(DecodeParams p) {
+  __shared__ int s_slot[kRanges];
+  __shared__ float s_w[kCombineHeads][kRanges];
   const int bt = blockIdx.x;
   const int nseg = p.bt_nseg[bt];
   if (nseg == 1) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * kCombineHeads + warp;
   const int first = p.bt_first[bt];
-  for (int hh = 0; hh < kCombineHeads; ++hh) {
-    const int h = blockIdx.y * kCombineHeads + hh;
-    if (h >= p.H) break;
-    float* dst = p.out + ((size_t)bt * p.H + h) * p.r;
-    if (nseg == 0) {
-      for (int d = threadIdx.x; d < p.r; d += blockDim.x) dst[d] = 0.f;
-      if (threadIdx.x == 0 && p.lse) p.lse[(size_t)bt * p.H + h] = -INFINITY;
-      continue;
-    }
-    float mx = -INFINITY;
-    for (int k = 0; k < nseg; ++k)
-      mx = fmaxf(mx, p.part_lse[(size_t)p.segments[first + k].slot * p.H + h]);
-    if (mx == -INFINITY) {  // every part empty (all its blocks were rejected): no rows
-      for (int d = threadIdx.x; d < p.r; d += blockDim.x) dst[d] = 0.f;
-      if (threadIdx.x == 0 && p.lse) p.lse[(size_t)bt * p.H + h] = -INFINITY;
-      continue;
-    }
-    float z = 0.f;
-    for (int k = 0; k < nseg; ++k)
-      z += expf(p.part_lse[(size_t)p.segments[first + k].slot * p.H + h] - mx);
-    const float L = mx + logf(z);
-    for (int d = threadIdx.x; d < p.r; d += blockDim.x) {
-      float acc = 0.f;
-      for (int k = 0; k < nseg; ++k) {
-        const int slot = p.segments[first + k].slot;
-        const float w = expf(p.part_lse[(size_t)slot * p.H + h] - L);
-        acc = fmaf(w, p.part_o[((size_t)slot * p.H + h) * p.r + d], acc);
-      }
-      dst[d] = acc;
-    }
-    if (threadIdx.x == 0 && p.lse) p.lse[(size_t)bt * p.H + h] = L;
+  for (int k = threadIdx.x; k < nseg; k += blockDim.x) s_slot[k] = p.segments[first + k].slot;
+  __syncthreads();
+  if (h >= p.H) return;
+  float4* dst = (float4*)(p.out + ((size_t)bt * p.H + h) * p.r);
+  const int r4 = p.r / 4;
+  float mx = -INFINITY;
+  for (int k = lane; k < nseg; k += 32) mx = fmaxf(mx, p.part_lse[(size_t)s_slot[k] * p.H + h]);
+  mx = warp_max(mx);
+  if (nseg == 0 || mx == -INFINITY) {  // no rows (bad length, or every block rejected)
+    for (int d = lane; d < r4; d += 32) dst[d] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane == 0 && p.lse) p.lse[(size_t)bt * p.H + h] = -INFINITY;
+    return;
   }
+  float z = 0.f;
+  for (int k = lane; k < nseg; k += 32) z += expf(p.part_lse[(size_t)s_slot[k] * p.H + h] - mx);
+  z = warp_sum(z);
+  const float L = mx + logf(z);
+  for (int k = lane; k < nseg; k += 32)
+    s_w[warp][k] = expf(p.part_lse[(size_t)s_slot[k] * p.H + h] - L);
+  __syncwarp();
+  for (int d = lane; d < r4; d += 32) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int k = 0; k < nseg; ++k) {
+      const float w = s_w[warp][k];
+      const float4 v = __ldcs((const float4*)(p.part_o + ((size_t)s_slot[k] * p.H + h) * p.r) + d);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    dst[d] = acc;
+  }
+  if (lane == 0 && p.lse) p.lse[(size_t)bt * p.H + h] = L;
 }
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t st) {

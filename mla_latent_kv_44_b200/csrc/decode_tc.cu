@@ -13,23 +13,23 @@
 // latent dims at a time. O for 128 heads x 512 dims in fp32 fills one SM's tensor memory, so
 // the two CTAs of a cluster take different roles for each work range:
 //   * the score CTA keeps the latent part of Q in TMEM (256 columns, A operand) and its RoPE
-//     part in shared memory, streams the cache rows' 64-dim slabs by TMA, accumulates S in the
-//     other 256 TMEM columns, runs the online softmax (exp2 units, O rescaled lazily only when
-//     the running max grows by more than 2^8) and sends P (bf16) with the per-row rescale
-//     factors and sums to the value CTA as 16 KB bulk copies into a 6-slot ring in its shared
-//     memory;
+//     part in shared memory, streams the cache rows' 64-dim slabs by TMA and accumulates S in
+//     the other 256 TMEM columns. Eight softmax warps copy S into registers (128 values per
+//     thread) and release it at once, so the next tile's S = Q . K^T runs on the tensor core
+//     while this tile's online softmax runs (exp2 units, O rescaled lazily only when the
+//     running max grows by more than 2^8). P (bf16) and the per-row rescale factors and sums
+//     go to the value CTA as 16 KB bulk copies into a 6-slot ring in its shared memory;
 //   * the value CTA streams the latent part of the same rows by TMA and accumulates O = P . V
 //     in its whole TMEM, applies rescales, and writes the normalised output.
 // The two read the same cache blocks close together in time, so HBM sees each row about once.
-// Warps: 0 TMA, 1 MMA issue, 2-5 softmax (score CTA) or rescale and epilogue (value CTA), 6
-// the cross-CTA traffic (bulk copies out of the score CTA, acknowledgements out of the value
-// CTA), so that no MMA-issuing warp ever waits on a cluster-scope fence.
+// Warps of the score CTA: 0 TMA, 1 MMA issue, 2-9 softmax, 10 bulk copies to the value CTA.
+// Warps of the value CTA: 0 TMA, 1 MMA issue, 2-5 rescale and epilogue, 6 acknowledgements to
+// the score CTA (7-10 idle). No MMA-issuing warp ever waits on a cluster-scope fence.
 // Every wait is bounded: on timeout the kernel sets MLA_DEV_WAIT_TIMEOUT, drains its copies
 // and MMAs, frees TMEM and returns. No TMA multicast is used.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "common.cuh"
+#include "tc_ptx.cuh"
+#include "tma_map.h"
 
 namespace mla {
 namespace {
@@ -41,7 +41,7 @@ constexpr int kD = kR + kDR;
 constexpr int kRows = 64;                       // rows per cache block = planner chunk
 constexpr int kTileBlocks = 4;                  // blocks per score tile (N <= 256)
 constexpr int kSlabBytes = kRows * 64 * 2;      // 64 rows x 64 dims bf16: 8 KB
-constexpr int kThreads = 224;  // 7 warps
+constexpr int kThreads = 352;  // 11 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kTimeoutNs = 1000000000ull;  // 1 s per wait
 
@@ -55,7 +55,8 @@ constexpr int kS_K = 0;
 constexpr int kS_QRope = kS_K + kKStages * kKStageBytes;      // 128 KB
 constexpr int kS_Stage = kS_QRope + kQRopeBytes;              // 144 KB
 constexpr int kS_Hdr = kS_Stage + kTileBlocks * kPBlockBytes; // 208 KB
-constexpr int kS_End = kS_Hdr + kHdrBytes;
+constexpr int kS_Red = kS_Hdr + kHdrBytes;                    // row max / sum exchange
+constexpr int kS_End = kS_Red + 4 * kH * 4;
 // value CTA: V stages (one block's 256-dim half), P ring, header ring
 constexpr int kVStages = 3;
 constexpr int kVStageBytes = 4 * kSlabBytes;                  // 32 KB
@@ -78,189 +79,25 @@ enum Bar {
   kStgFree,                     // value CTA received the previous tile's P (staging reusable)
   kStaged,                      // softmax warps finished writing a tile's P and header
   kSlotFree,                    // kPSlots: value CTA finished with a P ring slot
+  kRedMax = kSlotFree + kPSlots,  // the 8 softmax warps posted their row maxima
+  kRedSum,                        // ... and their row sums
   // value CTA
-  kVFull = kSlotFree + kPSlots,
+  kVFull = kRedSum + 1,
   kVEmpty = kVFull + kVStages,
   kPFull = kVEmpty + kVStages,  // kPSlots
   kHFull = kPFull + kPSlots,    // kHdrSlots
   kSlotDone = kHFull + kHdrSlots,  // kPSlots: P . V MMAs reading a slot are complete
   kOReady = kSlotDone + kPSlots,   // rescale (if any) applied, previous epilogue done
   kPvDone,                         // 2: all P . V of a tile complete (even / odd tiles)
-  kFinal = kPvDone + 2,
+  kHdrRead = kPvDone + 2,          // the 4 epilogue warps have read a header slot
+  kFinal,
   kNumBars
 };
 constexpr int kBarOff = kDataBytes;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;  // +1024: manual alignment
 
-// instruction descriptors, kind::f16: bf16 A and B, fp32 D, A K-major
-__host__ __device__ constexpr uint32_t idesc(int M, int N, int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
 constexpr uint32_t kIdescPV = idesc(128, 256, 1);
 
-// ------------------------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ uint32_t saddr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t peer_addr(uint32_t a, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
-               ::: "memory");
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                         int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y)
-      : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-// D[tmem] (+)= A[tmem] . B[smem]
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t id,
-                                       uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d), "r"(a), "l"(bdesc),
-      "r"(id), "r"(acc)
-      : "memory");
-}
-// 32 consecutive columns of this thread's TMEM lane, waited before returning.
-__device__ __forceinline__ void tmem_ld32(uint32_t ta, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
-        "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
-        "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(ta)
-      : "memory");
-}
-// 64 consecutive columns, one wait.
-__device__ __forceinline__ void tmem_ld64(uint32_t ta, uint32_t (&v)[64]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,"
-      "%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
-        "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
-        "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31]), "=r"(v[32]), "=r"(v[33]), "=r"(v[34]),
-        "=r"(v[35]), "=r"(v[36]), "=r"(v[37]), "=r"(v[38]), "=r"(v[39]), "=r"(v[40]), "=r"(v[41]),
-        "=r"(v[42]), "=r"(v[43]), "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47]), "=r"(v[48]),
-        "=r"(v[49]), "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]), "=r"(v[55]),
-        "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]), "=r"(v[61]), "=r"(v[62]),
-        "=r"(v[63])
-      : "r"(ta), "r"(ta + 32u)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st32(uint32_t ta, const uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(ta),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
-      "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]),
-      "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]),
-      "r"(v[30]), "r"(v[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Shared-memory matrix descriptor (Blackwell version 1): start, leading and stride byte
-// offsets in 16-byte units, swizzle mode in bits 61-63 (2 = 128-byte, 4 = 64-byte).
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo,
-                                          uint32_t swz) {
-  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | ((uint64_t)swz << 61);
-}
-
-// D[tmem] (+)= A[smem] . B[smem]
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t id,
-                                       uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d), "l"(adesc),
-      "l"(bdesc), "r"(id), "r"(acc)
-      : "memory");
-}
-// shared::cta -> peer shared::cluster bulk copy, completing bytes on the peer's mbarrier
-__device__ __forceinline__ void bulk_to_peer(uint32_t dst, uint32_t src, uint32_t bytes,
-                                             uint32_t peer_bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(dst), "r"(src), "r"(bytes), "r"(peer_bar)
-      : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_peer(uint32_t bar_in_peer) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_in_peer)
-               : "memory");
-}
-// the four softmax / epilogue warps (threads 64..191)
-__device__ __forceinline__ void sync_math_warps() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-}
 
 struct Ctl {
   uint32_t* err;
@@ -284,6 +121,15 @@ __device__ __noinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Ctl&
       return false;
     }
   }
+}
+
+// Barrier of a group of warps on an mbarrier that counts one arrival per warp: the k-th use
+// (k = 0, 1, ...) waits for parity k & 1. Bounded like every other wait, so a warp that gave
+// up elsewhere cannot leave the rest of its group blocked.
+__device__ __forceinline__ bool group_sync(uint32_t bar, int k, const Ctl& c) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  return warp_wait(bar, (uint32_t)k & 1u, c);
 }
 
 // Bounded wait for a phase that normally completed long ago (drains at teardown).
@@ -343,7 +189,7 @@ __device__ __forceinline__ int tile_block(const DecodeParams& p, const Tile& tl,
 
 }  // namespace
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(168)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
                  const __grid_constant__ CUtensorMap tm_q, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -366,13 +212,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
         mbar_init(bar(kKFull + i), 1);
         mbar_init(bar(kKEmpty + i), 1);
       }
-      mbar_init(bar(kQFull), 5);
+      mbar_init(bar(kQFull), 9);
       mbar_init(bar(kQEmpty), 1);
       mbar_init(bar(kSFull), 1);
-      mbar_init(bar(kSFree), 4);
+      mbar_init(bar(kSFree), 8);
       mbar_init(bar(kStgFree), 1);
-      mbar_init(bar(kStaged), 4);
+      mbar_init(bar(kStaged), 8);
       for (int i = 0; i < kPSlots; ++i) mbar_init(bar(kSlotFree + i), 1);
+      mbar_init(bar(kRedMax), 8);
+      mbar_init(bar(kRedSum), 8);
     } else {
       for (int i = 0; i < kVStages; ++i) {
         mbar_init(bar(kVFull + i), 1);
@@ -386,6 +234,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       mbar_init(bar(kOReady), 4);
       mbar_init(bar(kPvDone), 1);
       mbar_init(bar(kPvDone + 1), 1);
+      mbar_init(bar(kHdrRead), 4);
       // every P slot and header slot expects one bulk copy from the score CTA per use
       for (int i = 0; i < kPSlots; ++i) mbar_expect_tx(bar(kPFull + i), kPBlockBytes);
       for (int i = 0; i < kHdrSlots; ++i) mbar_expect_tx(bar(kHFull + i), kHdrBytes);
@@ -492,20 +341,25 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       __syncwarp();
       ++t;
     }
-  } else if (score && warp < 6) {
+  } else if (score && warp >= 2 && warp < 10) {
     // ---------------------------------------------------------------- score: softmax, P staged
+    // Eight warps: warp w reads TMEM lanes 32 * (w % 4) (its heads) and S columns
+    // 128 * half .. +127 (two cache blocks). S is copied into registers at once and released,
+    // so the MMA warp computes the next tile's S while this tile's softmax runs.
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int h = quad * 32 + lane;
     const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
     const float c2 = p.scale * 1.4426950408889634f;  // scores in log2 units
     const __nv_bfloat16* Q = (const __nv_bfloat16*)p.q;
     const uint32_t stage_p = s_base + kS_Stage;
     const uint32_t hdr = s_base + kS_Hdr;
+    float* red = (float*)(smem + kS_Red);  // [0..255]: max of half 0 / 1; [256..511]: sums
 
-    auto load_qckv = [&](int bt) {  // latent part of Q into TMEM columns [256, 512)
+    auto load_qckv = [&](int bt) {  // this warp's half of Q's latent part into TMEM
       const uint4* src = (const uint4*)(Q + ((size_t)bt * kH + h) * kD);
 #pragma unroll 1
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int ch = 4 * half; ch < 4 * half + 4; ++ch) {
         uint32_t w[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -520,7 +374,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       if (lane == 0) mbar_arrive(bar(kQFull));
     };
 
-    int t = 0, g = 0;
+    int t = 0;
     float m_ref = 0.f, l = 0.f;
     bool ok = true, q_loaded = false;
     while (ok && walk.next(tl)) {
@@ -530,18 +384,25 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       }
       if (!warp_wait(bar(kSFull), t & 1, ctl)) break;
       tc_after();
-      // pass 1: row max over the tile's valid rows
-      float mt = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < tl.nb; ++c) {
-        uint32_t v[64];
-        tmem_ld64(tq + 64 * c, v);
-        const int lim = tl.ntok - 64 * c;
-#pragma unroll
-        for (int k = 0; k < 64; ++k)
-          if (k < lim) mt = fmaxf(mt, __uint_as_float(v[k]));
+      uint32_t v[128];
+      tmem_ld128(tq + 128 * half, v);
+      tc_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kSFree));  // the next tile's S may be computed now
+      if (tl.last) {  // the segment's last S product is done: bring in the next query
+        TileWalk look = walk;
+        Tile nx;
+        if (look.next(nx)) load_qckv(nx.bt);
       }
-      mt *= c2;
+      // pass 1: row max over the valid rows of both halves
+      const int lim = tl.ntok - 128 * half;
+      float mt = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 128; ++k)
+        if (k < lim) mt = fmaxf(mt, __uint_as_float(v[k]));
+      red[half * kH + h] = mt;
+      if (!group_sync(bar(kRedMax), t, ctl)) break;
+      mt = fmaxf(red[h], red[kH + h]) * c2;
       float alpha = 1.f;
       if (tl.first) {
         m_ref = mt;
@@ -552,55 +413,50 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       }
       // the value CTA must have received the previous tile before staging is overwritten
       if (t > 0 && !warp_wait(bar(kStgFree), (t - 1) & 1, ctl)) break;
-      // pass 2: P = exp2(s * c2 - m_ref), rounded to bf16, into the A-operand layout
+      // pass 2: P = exp2(s * c2 - m_ref), rounded to bf16, packed in place, into the A-operand
+      // layout of the value CTA's P . V (K-major, 128-byte rows swizzled by row % 8)
       float rs = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < tl.nb; ++c) {
-        uint32_t v[64];
-        tmem_ld64(tq + 64 * c, v);
-        const int lim = tl.ntok - 64 * c;
-        uint32_t pw[32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float p0 = (2 * k < lim) ? ex2(__uint_as_float(v[2 * k]) * c2 - m_ref) : 0.f;
-          const float p1 = (2 * k + 1 < lim) ? ex2(__uint_as_float(v[2 * k + 1]) * c2 - m_ref) : 0.f;
-          rs += p0;
-          rs += p1;
-          pw[k] = pack_bf16(p0, p1);
-        }
-        const uint32_t row = stage_p + c * kPBlockBytes + (uint32_t)h * 128;
+      for (int k = 0; k < 64; ++k) {
+        const float p0 = (2 * k < lim) ? ex2(__uint_as_float(v[2 * k]) * c2 - m_ref) : 0.f;
+        const float p1 = (2 * k + 1 < lim) ? ex2(__uint_as_float(v[2 * k + 1]) * c2 - m_ref) : 0.f;
+        rs += p0;
+        rs += p1;
+        v[k] = pack_bf16(p0, p1);
+      }
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb) {
+        const uint32_t row = stage_p + (2 * half + cb) * kPBlockBytes + (uint32_t)h * 128;
 #pragma unroll
         for (int u = 0; u < 8; ++u)
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
                            row + 16u * (uint32_t)(u ^ (h & 7))),
-                       "r"(pw[4 * u]), "r"(pw[4 * u + 1]), "r"(pw[4 * u + 2]), "r"(pw[4 * u + 3])
+                       "r"(v[32 * cb + 4 * u]), "r"(v[32 * cb + 4 * u + 1]),
+                       "r"(v[32 * cb + 4 * u + 2]), "r"(v[32 * cb + 4 * u + 3])
                        : "memory");
       }
-      l = l * alpha + rs;
-      tc_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kSFree));  // S may be overwritten by the next tile
-      asm volatile("st.shared.f32 [%0], %1;" ::"r"(hdr + 4u * h), "f"(alpha) : "memory");
-      if (tl.last) asm volatile("st.shared.f32 [%0], %1;" ::"r"(hdr + 4u * (kH + h)), "f"(l) : "memory");
+      red[2 * kH + half * kH + h] = rs;
+      if (!group_sync(bar(kRedSum), t, ctl)) break;
+      if (half == 0) {
+        rs += red[3 * kH + h];
+        l = l * alpha + rs;
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(hdr + 4u * h), "f"(alpha) : "memory");
+        if (tl.last) asm volatile("st.shared.f32 [%0], %1;" ::"r"(hdr + 4u * (kH + h)), "f"(l) : "memory");
+      }
       fence_proxy_async();  // staged bytes are read by the bulk copies (async proxy)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kStaged));
-      if (tl.last) {
+      if (tl.last && half == 0) {
         const float lse = (m_ref + __log2f(l)) * 0.6931471805599453f;
         if (tl.slot < 0) {
           if (p.lse) p.lse[(size_t)tl.bt * kH + h] = lse;
         } else {
           p.part_lse[(size_t)tl.slot * kH + h] = lse;
         }
-        // the next segment's query: this segment's last S product is complete
-        TileWalk look = walk;
-        Tile nx;
-        if (look.next(nx)) load_qckv(nx.bt);
       }
-      g += tl.nb;
       ++t;
     }
-  } else if (score && warp == 6) {
+  } else if (score && warp == 10) {
     // ---------------------------------------------------------------- score: ship P out
     const uint32_t peer_slots = peer_addr(s_base + kV_P, peer);
     const uint32_t peer_hdr = peer_addr(s_base + kV_Hdr, peer);
@@ -731,7 +587,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       __syncwarp();
       ++t;
     }
-  } else {
+  } else if (!score && warp >= 2 && warp < 6) {
     // ---------------------------------------------------------------- value: rescale, epilogue
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
@@ -757,7 +613,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       float alpha;
       asm volatile("ld.shared.f32 %0, [%1];" : "=f"(alpha) : "r"(hb + 4u * h) : "memory");
       if (tl.last) asm volatile("ld.shared.f32 %0, [%1];" : "=f"(l_last) : "r"(hb + 4u * (kH + h)) : "memory");
-      sync_math_warps();  // everyone has read the header before it is re-armed
+      if (!group_sync(bar(kHdrRead), t, ctl)) break;  // all read it before it is re-armed
       if (threadIdx.x == 64) mbar_expect_tx(bar(kHFull + hs), kHdrBytes);
       if (!tl.first && __any_sync(0xffffffffu, alpha != 1.f)) {
         if (!wait_pv(t - 1)) break;
@@ -817,36 +673,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
   cluster_sync();  // the peer no longer touches this CTA's shared memory
 }
 
-namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// 2-D bf16 view [rows][576] with 128-byte swizzled boxes of 64 columns x box_rows rows.
-bool make_map(CUtensorMap* m, const void* base, long long rows, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
-
 bool tc_supported(const mla_config& c) {
   return c.dtype == MLA_BF16 && c.num_heads == kH && c.kv_rank == kR && c.rope_dim == kDR &&
          c.block_size == kRows;
@@ -855,8 +681,8 @@ bool tc_supported(const mla_config& c) {
 cudaError_t launch_attend_tc(const mla_config& c, const DecodeParams& p, cudaStream_t st) {
   (void)c;
   CUtensorMap kv, qm;
-  if (!make_map(&kv, p.pool, (long long)p.num_blocks * kRows, kRows) ||
-      !make_map(&qm, p.q, (long long)p.BT * kH, kH))
+  if (!make_bf16_map(&kv, p.pool, kD, (uint64_t)p.num_blocks * kRows, kD * 2, kRows) ||
+      !make_bf16_map(&qm, p.q, kD, (uint64_t)p.BT * kH, kD * 2, kH))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {

@@ -49,12 +49,18 @@ int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
 
 mla_status mla_absorb_query(const mla_config* cfg, const void* q_nope, const void* q_rope,
                             const int32_t* pos, const void* w_uk, void* q_out, int32_t n_tokens,
-                            void* stream) {
+                            uint32_t* dev_err, void* stream) {
   if (!valid_config(cfg) || n_tokens < 0) return MLA_ERR_INVALID_ARG;
   if (n_tokens == 0) return MLA_OK;
   if (!q_nope || !w_uk || !q_out || !pos || (cfg->rope_dim > 0 && !q_rope))
     return MLA_ERR_INVALID_ARG;
   if (n_tokens > (1 << 24)) return MLA_ERR_UNSUPPORTED;
+  const bool tc = cfg->decode_kernel != MLA_DECODE_SIMT && absorb_tc_supported(*cfg) &&
+                  aligned(q_nope, 16) && aligned(w_uk, 16);
+  if (cfg->decode_kernel == MLA_DECODE_TENSOR && !tc) return MLA_ERR_UNSUPPORTED;
+  if (tc)
+    return from_cuda(launch_absorb_tc(*cfg, q_nope, q_rope, pos, w_uk, q_out, n_tokens, dev_err,
+                                      (cudaStream_t)stream));
   return from_cuda(launch_absorb(*cfg, q_nope, q_rope, pos, w_uk, q_out, n_tokens,
                                  (cudaStream_t)stream));
 }
@@ -99,7 +105,8 @@ mla_status mla_decode_stages(const mla_config* cfg, int32_t stages, const void* 
   const size_t need = mla_decode_workspace_size(cfg, batch, q_per_seq);
   if (need == 0) return MLA_ERR_INVALID_ARG;
   if (workspace_bytes < need || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
-  if (!aligned(pool, 16) || !aligned(q, 16)) return MLA_ERR_INVALID_ARG;
+  if (!aligned(pool, 16) || !aligned(q, 16) || !aligned(out_latent, 16))
+    return MLA_ERR_INVALID_ARG;
 
   bool use_tc;
   switch (cfg->decode_kernel) {
@@ -162,11 +169,17 @@ mla_status mla_decode(const mla_config* cfg, const void* q, const void* pool,
 }
 
 mla_status mla_output(const mla_config* cfg, const float* out_latent, const void* w_uv, void* o,
-                      int32_t n_tokens, void* stream) {
+                      int32_t n_tokens, uint32_t* dev_err, void* stream) {
   if (!valid_config(cfg) || n_tokens < 0) return MLA_ERR_INVALID_ARG;
   if (n_tokens == 0) return MLA_OK;
   if (!out_latent || !w_uv || !o) return MLA_ERR_INVALID_ARG;
   if (n_tokens > (1 << 24)) return MLA_ERR_UNSUPPORTED;
+  const bool tc = cfg->decode_kernel != MLA_DECODE_SIMT && output_tc_supported(*cfg) &&
+                  aligned(out_latent, 16) && aligned(w_uv, 16);
+  if (cfg->decode_kernel == MLA_DECODE_TENSOR && !tc) return MLA_ERR_UNSUPPORTED;
+  if (tc)
+    return from_cuda(launch_output_tc(*cfg, out_latent, w_uv, o, n_tokens, dev_err,
+                                      (cudaStream_t)stream));
   return from_cuda(launch_output(*cfg, out_latent, w_uv, o, n_tokens, (cudaStream_t)stream));
 }
 

@@ -10,7 +10,7 @@ namespace mla {
 
 // ------------------------------------------------------------------------------------------
 // Absorbed query: Q[n,h,:r] = W_UK[h]^T q_nope[n,h];  Q[n,h,r:] = RoPE(q_rope[n,h], pos[n]).
-// One CTA per (head, 16 tokens); thread j owns latent columns j, j+256, ... of W_UK[h], which
+// One CTA per (16 tokens, head); thread j owns latent columns j, j+256, ... of W_UK[h], which
 // it streams row by row (coalesced across the CTA) while the 16 query rows sit in shared memory.
 // ------------------------------------------------------------------------------------------
 constexpr int kAbsorbTokens = 16;
@@ -21,8 +21,8 @@ absorb_kernel(const T* __restrict__ q_nope, const T* __restrict__ q_rope,
               const int32_t* __restrict__ pos, const T* __restrict__ w_uk, T* __restrict__ q_out,
               int n, int H, int dh, int r, int dr, float base) {
   extern __shared__ float s_q[];  // kAbsorbTokens x dh
-  const int h = blockIdx.x;
-  const int n0 = blockIdx.y * kAbsorbTokens;
+  const int h = blockIdx.y;
+  const int n0 = blockIdx.x * kAbsorbTokens;
   const int nt = min(kAbsorbTokens, n - n0);
   for (int idx = threadIdx.x; idx < kAbsorbTokens * dh; idx += blockDim.x) {
     const int t = idx / dh, i = idx - t * dh;
@@ -85,7 +85,7 @@ static cudaError_t absorb_go(const mla_config& c, const void* qn, const void* qr
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(c.num_heads, (n + kAbsorbTokens - 1) / kAbsorbTokens);
+  dim3 grid((n + kAbsorbTokens - 1) / kAbsorbTokens, c.num_heads);
   k<<<grid, 256, smem, st>>>((const T*)qn, (const T*)qr, pos, (const T*)w, (T*)q, n, c.num_heads,
                              c.head_dim, c.kv_rank, c.rope_dim, c.rope_base);
   return cudaGetLastError();
@@ -172,7 +172,7 @@ cudaError_t launch_append(const mla_config& c, const void* ckv, const void* kr,
 }
 
 // ------------------------------------------------------------------------------------------
-// Output: o[n,h,i] = sum_j W_UV[h,i,j] * lat[n,h,j]. One CTA per (head, 16 tokens); each warp
+// Output: o[n,h,i] = sum_j W_UV[h,i,j] * lat[n,h,j]. One CTA per (16 tokens, head); each warp
 // streams whole rows of W_UV[h] (coalesced) against the 16 latent rows held in shared memory.
 // ------------------------------------------------------------------------------------------
 constexpr int kOutTokens = 16;
@@ -182,8 +182,8 @@ __global__ void __launch_bounds__(256)
 output_kernel(const float* __restrict__ lat, const T* __restrict__ w_uv, T* __restrict__ o, int n,
               int H, int dv, int r) {
   extern __shared__ float s_lat[];  // kOutTokens x r
-  const int h = blockIdx.x;
-  const int n0 = blockIdx.y * kOutTokens;
+  const int h = blockIdx.y;
+  const int n0 = blockIdx.x * kOutTokens;
   const int nt = min(kOutTokens, n - n0);
   for (int idx = threadIdx.x; idx < kOutTokens * r; idx += blockDim.x) {
     const int t = idx / r, j = idx - t * r;
@@ -212,7 +212,7 @@ output_kernel(const float* __restrict__ lat, const T* __restrict__ w_uv, T* __re
 cudaError_t launch_output(const mla_config& c, const float* lat, const void* w_uv, void* o,
                           int n, cudaStream_t st) {
   const size_t smem = sizeof(float) * kOutTokens * c.kv_rank;
-  dim3 grid(c.num_heads, (n + kOutTokens - 1) / kOutTokens);
+  dim3 grid((n + kOutTokens - 1) / kOutTokens, c.num_heads);
   if (c.dtype == MLA_BF16) {
     auto k = output_kernel<__nv_bfloat16>;
     if (smem > 48 * 1024)

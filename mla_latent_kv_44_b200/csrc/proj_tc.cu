@@ -1,0 +1,416 @@
+// tcgen05 tensor-core projections of the bf16 decode step, for sm_100a:
+//   absorbed query   Q[n, h, 0:r] = W_UK[h]^T q_nope[n, h]        ("DeepSeek MLA, Built From the
+//                    Paper", 3 Matrix absorption: W_UK folds into the query)
+//   output           o[n, h, :]   = W_UV[h] o_lat[n, h, :]         ("MLA from scratch in
+//                    PyTorch", Absorbing projections: W_UV after the weighted sum)
+// Per head both are small dense GEMMs whose cost is reading the weights once (16.8 MB each at
+// H = 128, d = 128, r = 512). The weight tile is the M = 128 side of the MMA (latent dims for
+// the query, output dims for the output), the tokens are its N side, so one CTA handles one
+// (head, 128-row weight tile, token tile): TMA brings the weight tile and the bf16 query rows
+// into shared memory in the 128-byte swizzled layout, one thread issues the MMAs into an fp32
+// TMEM accumulator, and four warps read it back and store bf16. The output's latent operand is
+// fp32 in memory; threads split it into two bf16 terms while writing it into the same
+// swizzled layout, so the MMA's operands are bf16, its sums fp32, and the latent keeps about
+// 16 significant bits.
+// Every mbarrier wait gives up after 1 s: it then sets MLA_DEV_WAIT_TIMEOUT, waits (also
+// bounded) for the copies and MMAs already issued, frees TMEM and returns without storing.
+#include <algorithm>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+#include "tma_map.h"
+
+namespace mla {
+namespace {
+
+constexpr unsigned long long kProjTimeoutNs = 1000000000ull;
+constexpr int kWRows = 128;        // weight rows per CTA = MMA M
+constexpr int kMaxTokTile = 128;   // tokens per CTA at most = MMA N (TMEM columns)
+constexpr uint32_t kProjTmemCols = 128;
+constexpr int kSlab = 64;          // bf16 elements per 128-byte swizzled row
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint32_t* err) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try(bar, parity)) {
+    if (globaltimer() - t0 > kProjTimeoutNs) {
+      set_error(err, MLA_DEV_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Teardown after a failed wait: give a phase that may still complete its last chance.
+__device__ void drain_bounded(uint32_t bar, uint32_t parity, uint32_t* err) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try(bar, parity))
+    if (globaltimer() - t0 > kProjTimeoutNs) {
+      set_error(err, MLA_DEV_WAIT_TIMEOUT);
+      return;
+    }
+}
+
+__device__ __forceinline__ uint32_t tmem_alloc_cols(uint32_t slot_addr) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_addr),
+               "r"(kProjTmemCols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  return 0;
+}
+__device__ __forceinline__ void tmem_free_cols(uint32_t tmem) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+               "r"(kProjTmemCols)
+               : "memory");
+}
+
+__host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// ------------------------------------------------------------------------------------------
+// Absorbed query. Grid (token tiles, ceil(r / 128), H); 128 threads.
+// Shared memory: A = W_UK[h][:, j0 : j0+128] as two MN-major slabs (64 latent dims x d_h rows
+// of 128 B each); B = q_nope[n0 : n0+tile, h, :] as d_h / 64 K-major slabs (tile rows x 128 B).
+// D[j, n] = sum_i A[j, i] B[i, n] lands in TMEM lane j, column n.
+// ------------------------------------------------------------------------------------------
+struct AbsorbArgs {
+  const __nv_bfloat16* q_rope;
+  const int32_t* pos;
+  __nv_bfloat16* q_out;
+  uint32_t* err;
+  int n, H, dh, r, dr, tile;
+  float base;
+};
+
+__global__ void __launch_bounds__(128)
+absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
+                 const AbsorbArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int jt = blockIdx.y, h = blockIdx.z, n0 = blockIdx.x * a.tile;
+  const int ntok = min(a.tile, a.n - n0);
+  const int nmma = round_up(ntok, 16);
+  const int ksl = a.dh / kSlab;                      // K slabs of the query rows
+  const uint32_t slab_a = (uint32_t)a.dh * 128;      // one 64-dim slab of the weight tile
+  const uint32_t slab_b = (uint32_t)round_up(a.tile * 128, 1024);
+  const uint32_t sA = saddr(smem);
+  const uint32_t sB = sA + 2 * slab_a;
+  uint8_t* ctl = smem + 2 * slab_a + ksl * slab_b;
+  const uint32_t bar_full = saddr(ctl), bar_done = bar_full + 8;
+  uint32_t* tmem_slot = (uint32_t*)(ctl + 16);
+  int* flags = (int*)(ctl + 32);  // [0] MMAs issued
+  const int j0 = jt * kWRows;
+  const int halves = (j0 + kSlab < a.r) ? 2 : 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_full, 1);
+    mbar_init(bar_done, 1);
+    flags[0] = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc_cols(saddr(tmem_slot));
+  tc_before();
+  __syncthreads();
+  tc_after();
+  const uint32_t tmem = *tmem_slot;
+
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(bar_full, halves * slab_a + ksl * (uint32_t)a.tile * 128);
+    for (int hf = 0; hf < halves; ++hf)
+      tma_load(sA + hf * slab_a, &tm_w, bar_full, j0 + kSlab * hf, h * a.dh);
+    for (int k = 0; k < ksl; ++k)
+      tma_load(sB + k * slab_b, &tm_q, bar_full, h * a.dh + kSlab * k, n0);
+  }
+
+  // RoPE part of the query, while the copies are in flight: pairs (2i, 2i+1) rotated by
+  // pos * base^(-2i/d_r), angle in double; the (token, pair) items of this head are dealt out
+  // over its gridDim.y CTAs
+  const int D = a.r + a.dr;
+  const int half = a.dr / 2;
+  for (int idx = jt * blockDim.x + threadIdx.x; idx < ntok * half; idx += gridDim.y * blockDim.x) {
+    const int t = idx / half, i = idx - t * half;
+    const int n = n0 + t;
+    double cs, sn;
+    rope_cos_sin(a.pos[n], i, a.dr, a.base, &cs, &sn);
+    const __nv_bfloat16* src = a.q_rope + ((size_t)n * a.H + h) * a.dr;
+    const double x0 = __bfloat162float(src[2 * i]), x1 = __bfloat162float(src[2 * i + 1]);
+    __nv_bfloat16* dst = a.q_out + ((size_t)n * a.H + h) * D + a.r;
+    dst[2 * i] = __float2bfloat16_rn((float)(x0 * cs - x1 * sn));
+    dst[2 * i + 1] = __float2bfloat16_rn((float)(x0 * sn + x1 * cs));
+  }
+
+  if (threadIdx.x == 0) {
+    ok = wait_bounded(bar_full, 0, a.err);
+    if (ok) {
+      tc_after();
+      const uint32_t id = idesc(kWRows, nmma, 0, 1);
+      for (int ks = 0; ks < a.dh / 16; ++ks) {
+        // A (MN-major): 16 K-rows further per step; LBO = distance of the two 64-dim slabs
+        const uint64_t ad = sdesc(sA + ks * 2048, slab_a, 1024, 2);
+        // B (K-major): 32 bytes further per step inside a slab, next slab every 4 steps
+        const uint64_t bd = sdesc(sB + (ks >> 2) * slab_b + (ks & 3) * 32, 16, 1024, 2);
+        mma_ss(tmem, ad, bd, id, ks > 0 ? 1u : 0u);
+      }
+      tc_commit(bar_done);
+      flags[0] = 1;
+    }
+  }
+  ok = __syncthreads_and(ok);
+  if (ok) ok = __syncthreads_and(wait_bounded(bar_done, 0, a.err));
+
+  if (ok) {
+    tc_after();
+    const int j = j0 + 32 * warp + lane;
+    for (int c0 = 0; c0 < nmma; c0 += 32) {
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + c0, v);
+      if (j < a.r) {
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) {
+          const int t = c0 + cc;
+          if (t < ntok)
+            a.q_out[((size_t)(n0 + t) * a.H + h) * D + j] = __float2bfloat16_rn(__uint_as_float(v[cc]));
+        }
+      }
+    }
+  }
+
+  tc_before();
+  __syncthreads();
+  tc_after();
+  if (!ok) {  // give in-flight copies and MMAs their chance to finish before freeing anything
+    if (threadIdx.x == 0) drain_bounded(bar_full, 0, a.err);
+    if (threadIdx.x == 32 && flags[0]) drain_bounded(bar_done, 0, a.err);
+    __syncthreads();
+  }
+  if (warp == 1) tmem_free_cols(tmem);
+}
+
+// ------------------------------------------------------------------------------------------
+// Output. Grid (token tiles, ceil(d_v / 128), H); 256 threads. The K = r contraction runs in
+// chunks of 128 latent dims through two shared-memory stages: TMA brings W_UV[h][i0:i0+128,
+// chunk] (K-major slabs of 128 rows x 128 B) while all threads write the chunk of o_lat as
+// bf16 K-major slabs (tile rows x 128 B, 16-byte groups XOR-swizzled by row % 8). The fp32
+// latent is split into two bf16 terms, hi = bf16(x) and lo = bf16(x - hi), and both are
+// multiplied by the (exactly bf16) weights, so the product sees x to about 16 significant
+// bits instead of bf16's 8.
+// D[i, n] = sum_j W[i, j] lat[n, j] lands in TMEM lane i, column n.
+// ------------------------------------------------------------------------------------------
+struct OutputArgs {
+  const float* lat;
+  __nv_bfloat16* o;
+  uint32_t* err;
+  int n, H, dv, r, tile;
+};
+
+__global__ void __launch_bounds__(256)
+output_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const OutputArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = blockIdx.y, h = blockIdx.z, n0 = blockIdx.x * a.tile;
+  const int ntok = min(a.tile, a.n - n0);
+  const int nmma = round_up(ntok, 16);
+  const int i0 = mt * kWRows;
+  constexpr uint32_t kSlabA = kWRows * 128;             // 16 KB
+  const uint32_t slab_b = (uint32_t)round_up(a.tile * 128, 1024);
+  const uint32_t stage_bytes = 2 * kSlabA + 4 * slab_b;  // W slabs, then hi and lo slabs
+  const uint32_t s0 = saddr(smem);
+  uint8_t* ctl = smem + 2 * stage_bytes;
+  const uint32_t bar_full = saddr(ctl);   // [2]
+  const uint32_t bar_done = bar_full + 16;  // [2]
+  uint32_t* tmem_slot = (uint32_t*)(ctl + 32);
+  int* flags = (int*)(ctl + 48);          // [0] chunks whose MMAs were committed, [1] loaded
+  const int nchunks = (a.r + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_done + 8 * s, 1);
+    }
+    flags[0] = 0;
+    flags[1] = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc_cols(saddr(tmem_slot));
+  tc_before();
+  __syncthreads();
+  tc_after();
+  const uint32_t tmem = *tmem_slot;
+
+  bool ok = true;
+  for (int c = 0; c < nchunks && ok; ++c) {
+    const int s = c & 1;
+    const uint32_t sA = s0 + s * stage_bytes, sB = sA + 2 * kSlabA;
+    uint8_t* pB = smem + s * stage_bytes + 2 * kSlabA;
+    const int k0 = c * 128;
+    const int width = min(128, a.r - k0);   // 64 or 128 (r is a multiple of 64)
+    const int nsl = width / kSlab;
+    if (c >= 2) {  // stage s is free once the MMAs of chunk c - 2 are done
+      ok = __syncthreads_and(wait_bounded(bar_done + 8 * s, ((c - 2) >> 1) & 1, a.err));
+      if (!ok) break;
+    }
+    if (threadIdx.x == 0) {
+      mbar_expect_tx(bar_full + 8 * s, nsl * kSlabA);
+      for (int k = 0; k < nsl; ++k)
+        tma_load(sA + k * kSlabA, &tm_w, bar_full + 8 * s, k0 + kSlab * k, h * a.dv + i0);
+      flags[1] = c + 1;
+    }
+    // o_lat chunk -> hi and lo bf16 terms, swizzled K-major: row t, 16-byte group g of slab
+    // k at g ^ (t & 7); the lo slabs follow the two hi slabs
+    const int groups = width / 8;
+    for (int idx = threadIdx.x; idx < a.tile * groups; idx += blockDim.x) {
+      const int t = idx / groups, q = idx - t * groups;
+      const int k = q >> 3, g = q & 7;
+      float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (t < ntok) {
+        const float4* src =
+            (const float4*)(a.lat + ((size_t)(n0 + t) * a.H + h) * a.r + k0 + 8 * q);
+        const float4 u = __ldg(src), v = __ldg(src + 1);
+        x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+        x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+      }
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
+        hi[e] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+        lo[e] = pack_bf16(x[2 * e] - __bfloat162float(h0), x[2 * e + 1] - __bfloat162float(h1));
+      }
+      const uint32_t off = k * slab_b + t * 128 + ((g ^ (t & 7)) << 4);
+      *(uint4*)(pB + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *(uint4*)(pB + 2 * slab_b + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      ok = wait_bounded(bar_full + 8 * s, (c >> 1) & 1, a.err);
+      if (ok) {
+        tc_after();
+        const uint32_t id = idesc(kWRows, nmma, 0, 0);
+        for (int ks = 0; ks < width / 16; ++ks) {
+          const uint64_t ad = sdesc(sA + (ks >> 2) * kSlabA + (ks & 3) * 32, 16, 1024, 2);
+          const uint32_t b_off = (ks >> 2) * slab_b + (ks & 3) * 32;
+          mma_ss(tmem, ad, sdesc(sB + b_off, 16, 1024, 2), id, (c > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(tmem, ad, sdesc(sB + 2 * slab_b + b_off, 16, 1024, 2), id, 1u);
+        }
+        tc_commit(bar_done + 8 * s);
+        flags[0] = c + 1;
+      }
+    }
+    ok = __syncthreads_and(ok);
+  }
+  const int last = nchunks - 1;
+  if (ok) ok = __syncthreads_and(wait_bounded(bar_done + 8 * (last & 1), (last >> 1) & 1, a.err));
+
+  if (ok) {
+    tc_after();
+    const int quad = warp & 3, colh = warp >> 2;
+    const int i = i0 + 32 * quad + lane;
+    for (int c0 = 64 * colh; c0 < min(nmma, 64 * colh + 64); c0 += 32) {
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + c0, v);
+      if (i < a.dv) {
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) {
+          const int t = c0 + cc;
+          if (t < ntok)
+            a.o[((size_t)(n0 + t) * a.H + h) * a.dv + i] = __float2bfloat16_rn(__uint_as_float(v[cc]));
+        }
+      }
+    }
+  }
+
+  tc_before();
+  __syncthreads();
+  tc_after();
+  if (!ok) {
+    const int committed = flags[0], loaded = flags[1];
+    // the copies of a chunk that never reached its MMAs, and the MMAs of the last commit
+    if (threadIdx.x == 0 && loaded > committed) {
+      const int c = loaded - 1;
+      drain_bounded(bar_full + 8 * (c & 1), (c >> 1) & 1, a.err);
+    }
+    if (threadIdx.x == 32 && committed > 0) {
+      const int c = committed - 1;
+      drain_bounded(bar_done + 8 * (c & 1), (c >> 1) & 1, a.err);
+    }
+    __syncthreads();
+  }
+  if (warp == 1) tmem_free_cols(tmem);
+}
+
+// Tokens per CTA: enough token tiles that the grid covers the 148 SMs about twice, each a
+// multiple of 16 (the MMA's N step) and at most 128 (the TMEM accumulator's columns).
+int token_tile(int n, int ctas_per_tile) {
+  const int want = (2 * 148 + ctas_per_tile - 1) / ctas_per_tile;
+  int tiles = (n + kMaxTokTile - 1) / kMaxTokTile;
+  tiles = std::max(tiles, std::min(want, (n + 15) / 16));
+  return std::min(kMaxTokTile, round_up((n + tiles - 1) / tiles, 16));
+}
+
+size_t absorb_smem(int dh, int tile) {
+  const size_t need = 1024 + 2 * (size_t)dh * 128 + (size_t)(dh / kSlab) * round_up(tile * 128, 1024) + 64;
+  // at least 61 KB: no more than three CTAs (3 x 128 TMEM columns) share an SM
+  return std::max(need, (size_t)61 * 1024);
+}
+
+size_t output_smem(int tile) {
+  const size_t stage = 2 * (size_t)kWRows * 128 + 4 * (size_t)round_up(tile * 128, 1024);
+  return std::max((size_t)1024 + 2 * stage + 64, (size_t)80 * 1024);
+}
+
+}  // namespace
+
+bool absorb_tc_supported(const mla_config& c) {
+  return c.dtype == MLA_BF16 && c.head_dim % kSlab == 0 && c.head_dim <= 256 &&
+         c.kv_rank % kSlab == 0 && c.rope_dim % 2 == 0;
+}
+
+bool output_tc_supported(const mla_config& c) {
+  return c.dtype == MLA_BF16 && c.kv_rank % kSlab == 0;
+}
+
+cudaError_t launch_absorb_tc(const mla_config& c, const void* q_nope, const void* q_rope,
+                             const int32_t* pos, const void* w_uk, void* q_out, int n,
+                             uint32_t* err, cudaStream_t st) {
+  const int H = c.num_heads, dh = c.head_dim, r = c.kv_rank;
+  const int jts = (r + kWRows - 1) / kWRows;
+  const int tile = token_tile(n, jts * H);
+  CUtensorMap tw, tq;
+  if (!make_bf16_map(&tw, w_uk, (uint64_t)r, (uint64_t)H * dh, (uint64_t)r * 2, (uint32_t)dh) ||
+      !make_bf16_map(&tq, q_nope, (uint64_t)H * dh, (uint64_t)n, (uint64_t)H * dh * 2,
+                     (uint32_t)tile))
+    return cudaErrorInvalidValue;
+  const size_t smem = absorb_smem(dh, tile);
+  cudaError_t e = cudaFuncSetAttribute(absorb_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  AbsorbArgs a{(const __nv_bfloat16*)q_rope, pos, (__nv_bfloat16*)q_out, err, n, H, dh, r,
+               c.rope_dim, tile, c.rope_base};
+  dim3 grid((n + tile - 1) / tile, jts, H);
+  absorb_tc_kernel<<<grid, 128, smem, st>>>(tw, tq, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_output_tc(const mla_config& c, const float* lat, const void* w_uv, void* o,
+                             int n, uint32_t* err, cudaStream_t st) {
+  const int H = c.num_heads, dv = c.head_dim_v, r = c.kv_rank;
+  const int mts = (dv + kWRows - 1) / kWRows;
+  const int tile = token_tile(n, mts * H);
+  if (((uintptr_t)lat & 15) != 0) return cudaErrorInvalidValue;
+  CUtensorMap tw;
+  if (!make_bf16_map(&tw, w_uv, (uint64_t)r, (uint64_t)H * dv, (uint64_t)r * 2, kWRows))
+    return cudaErrorInvalidValue;
+  const size_t smem = output_smem(tile);
+  cudaError_t e = cudaFuncSetAttribute(output_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  OutputArgs a{lat, (__nv_bfloat16*)o, err, n, H, dv, r, tile};
+  dim3 grid((n + tile - 1) / tile, mts, H);
+  output_tc_kernel<<<grid, 256, smem, st>>>(tw, a);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -130,7 +130,8 @@ class DecodeState:
 
     # ---- the hot path -------------------------------------------------------------------
     def absorb(self, stream=None):
-        absorb_query(self.cfg, self.q_nope, self.q_rope, self.pos_new, self.w_uk, self.q, stream)
+        absorb_query(self.cfg, self.q_nope, self.q_rope, self.pos_new, self.w_uk, self.q, stream,
+                     self.dev_err)
 
     def append(self, stream=None):
         append_latent(self.cfg, self.ckv_new, self.krope_new, self.gamma, self.seq_new,
@@ -141,7 +142,7 @@ class DecodeState:
                self.workspace, self.out_latent, self.lse, self.dev_err, stream, stages)
 
     def project(self, stream=None):
-        output(self.cfg, self.out_latent, self.w_uv, self.o, stream)
+        output(self.cfg, self.out_latent, self.w_uv, self.o, stream, self.dev_err)
 
     def step(self, stream=None):
         self.absorb(stream)

@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(mla):
 
 
 def test_abi_version_and_status_strings(mla):
-    assert mla.abi_version() == 1
+    assert mla.abi_version() == 2
     assert mla.status_string(0) == "MLA_OK"
     assert mla.status_string(4) == "MLA_ERR_WORKSPACE"
     assert mla.status_string(99) == "MLA_ERR_UNKNOWN"
@@ -69,14 +69,14 @@ def test_invalid_config_rejected(mla, bad):
     c = cfg.c()
     if bad.get("dtype") == "f16":
         c.dtype = 7
-    st = mla.lib.mla_absorb_query(ctypes.byref(c), 1, 1, 1, 1, 1, 4, None)
+    st = mla.lib.mla_absorb_query(ctypes.byref(c), 1, 1, 1, 1, 1, 4, None, None)
     assert st == mla.MLA_ERR_INVALID_ARG
 
 
 def test_null_pointers_rejected_without_launch(mla):
     c = _cfg(mla)
-    assert mla.lib.mla_absorb_query(ctypes.byref(c), None, 1, 1, 1, 1, 4, None) == 1
-    assert mla.lib.mla_output(ctypes.byref(c), None, 1, 1, 4, None) == 1
+    assert mla.lib.mla_absorb_query(ctypes.byref(c), None, 1, 1, 1, 1, 4, None, None) == 1
+    assert mla.lib.mla_output(ctypes.byref(c), None, 1, 1, 4, None, None) == 1
     assert mla.lib.mla_append_latent(ctypes.byref(c), 1, 1, 1, 1, 1, 1, 2, 2, 1, 4, 8, None,
                                      None) == 1
     ws = mla.lib.mla_decode_workspace_size(ctypes.byref(c), 2, 1)
@@ -94,8 +94,8 @@ def test_workspace_too_small_or_misaligned(mla):
 
 def test_empty_work_is_a_no_op(mla):
     c = _cfg(mla)
-    assert mla.lib.mla_absorb_query(ctypes.byref(c), None, None, None, None, None, 0, None) == 0
-    assert mla.lib.mla_output(ctypes.byref(c), None, None, None, 0, None) == 0
+    assert mla.lib.mla_absorb_query(ctypes.byref(c), None, None, None, None, None, 0, None, None) == 0
+    assert mla.lib.mla_output(ctypes.byref(c), None, None, None, 0, None, None) == 0
     assert mla.lib.mla_decode(ctypes.byref(c), None, None, None, 1, 1, None, 0, 1, None, 0, None,
                               None, None, None) == 0
 

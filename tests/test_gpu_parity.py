@@ -99,30 +99,44 @@ def test_full_step_large(mla, name):
 # Stage: absorbed query
 # ----------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("dtype,shape", [("f32", (16, 64, 64, 32)), ("bf16", (16, 64, 64, 32)),
-                                         ("bf16", (128, 128, 512, 64))])
-def test_absorb_stage(mla, dtype, shape):
+_SIMT, _TC = 1, 2  # mla_config.decode_kernel: CUDA-core or tensor-core kernels
+
+
+@pytest.mark.parametrize("dtype,shape,N,kernel", [
+    ("f32", (16, 64, 64, 32), 37, 0),
+    ("f32", (8, 32, 64, 16), 1, 0),
+    ("bf16", (16, 64, 64, 32), 37, _SIMT),
+    ("bf16", (16, 64, 64, 32), 37, _TC),
+    ("bf16", (128, 128, 512, 64), 37, _SIMT),
+    ("bf16", (128, 128, 512, 64), 1, _TC),
+    ("bf16", (128, 128, 512, 64), 64, _TC),
+    ("bf16", (128, 128, 512, 64), 200, _TC),
+    ("bf16", (4, 256, 192, 0), 300, _TC),
+])
+def test_absorb_stage(mla, dtype, shape, N, kernel):
     H, dh, r, dr = shape
-    N = 37
-    g = np.random.default_rng([1, 1])
+    g = np.random.default_rng([1, 1, N])
     qn = _store(g.standard_normal((N, H, dh)), dtype)
     qr = _store(g.standard_normal((N, H, dr)), dtype)
     wuk = _store(g.standard_normal((H, dh, r)) / math.sqrt(r), dtype)
     pos = g.integers(0, 32768, N).astype(np.int32)
-    pos[:3] = [0, 1, 32767]
+    pos[:min(N, 3)] = [0, 1, 32767][:min(N, 3)]
     dev = "cuda"
     t = _tdt(dtype)
     out = torch.empty((N, H, r + dr), dtype=t, device=dev)
-    cfg = _cfg(mla, H, dh, r, dr, 64, dtype)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    cfg = _cfg(mla, H, dh, r, dr, 64, dtype, kernel)
     mla.absorb_query(cfg, torch.from_numpy(qn).to(dev, t), torch.from_numpy(qr).to(dev, t),
-                     torch.from_numpy(pos).to(dev), torch.from_numpy(wuk).to(dev, t), out)
+                     torch.from_numpy(pos).to(dev), torch.from_numpy(wuk).to(dev, t), out,
+                     dev_err=err)
     got = out.float().cpu().numpy()
+    assert int(err.item()) == 0
     exp = ref.absorb_ref(qn, qr, pos, wuk, 10000.0)
     if dtype == "f32":
         assert compare.normwise_rel_error(got, exp) <= 1e-5
     else:
         # one bf16 rounding (relative u = 2^-8) of an fp32 sum of d_h products, whose own error
-        # is at most d_h * 2^-24 * sum |q_i w_ij|
+        # is at most d_h * 2^-24 * sum |q_i w_ij|, whatever order the kernel sums in
         u = 2.0 ** -8
         mag = ref.absorb_ref(np.abs(qn), np.abs(qr), np.zeros(N, np.int64), np.abs(wuk), 10000.0)
         bound = u * np.abs(exp) + 1.01 * dh * 2.0 ** -24 * mag + 1e-30
@@ -340,23 +354,43 @@ def test_decode_flags_bad_lengths_and_blocks(mla):
 # Stage: output projection
 # ----------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("dtype,shape", [("f32", (8, 32, 64)), ("bf16", (128, 128, 512))])
-def test_output_stage(mla, dtype, shape):
+@pytest.mark.parametrize("dtype,shape,N,kernel", [
+    ("f32", (8, 32, 64), 21, 0),
+    ("bf16", (128, 128, 512), 21, _SIMT),
+    ("bf16", (128, 128, 512), 1, _TC),
+    ("bf16", (128, 128, 512), 64, _TC),
+    ("bf16", (128, 128, 512), 200, _TC),
+    ("bf16", (16, 64, 64), 8, _TC),
+    ("bf16", (8, 32, 64), 21, _TC),
+    ("bf16", (2, 200, 320), 150, _TC),
+])
+def test_output_stage(mla, dtype, shape, N, kernel):
     H, dv, r = shape
-    N = 21
-    g = np.random.default_rng([1, 6])
+    g = np.random.default_rng([1, 6, N])
     lat = g.standard_normal((N, H, r)).astype(np.float32) * 0.05
     wuv = _store(g.standard_normal((H, dv, r)) / math.sqrt(r), dtype)
     t = _tdt(dtype)
     o = torch.empty((N, H, dv), dtype=t, device="cuda")
-    cfg = _cfg(mla, H, dv, r, 0, 64, dtype)
-    mla.output(cfg, torch.from_numpy(lat).cuda(), torch.from_numpy(wuv).to("cuda", t), o)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cfg = _cfg(mla, H, dv, r, 0, 64, dtype, kernel)
+    mla.output(cfg, torch.from_numpy(lat).cuda(), torch.from_numpy(wuv).to("cuda", t), o,
+               dev_err=err)
     got = o.float().cpu().numpy()
+    assert int(err.item()) == 0
     exp = ref.output_ref(lat, wuv)
     if dtype == "f32":
         assert compare.normwise_rel_error(got, exp) <= 1e-5
-    else:
-        assert compare.normwise_rel_error(got, exp) <= 2.0 ** -7
+        return
+    # bf16: an fp32 sum of r products (error <= r * 2^-24 * sum |w_ij lat_j|) rounded once to
+    # bf16 (relative u = 2^-8). The tensor-core kernel feeds the latent to its bf16 MMA as
+    # hi + lo (hi = bf16(x), lo = bf16(x - hi)), which misses x by at most 2^-16 |x| and sums
+    # 2r products instead of r.
+    u = 2.0 ** -8
+    mag = ref.output_ref(np.abs(lat), np.abs(wuv))
+    operand, terms = (2.0 ** -16, 2 * r) if kernel == _TC else (0.0, r)
+    bound = u * np.abs(exp) + (1 + u) * (operand + 1.02 * terms * 2.0 ** -24) * mag + 1e-30
+    ok = np.abs(got - exp) <= bound
+    assert ok.all(), f"{(~ok).sum()} of {ok.size} values outside the bound"
 
 
 def test_empty_calls_launch_nothing(mla):
