@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "mla.h"
 
 namespace mla {
@@ -112,6 +114,30 @@ __device__ __forceinline__ void rope_cos_sin(int p, int i, int dr, float base, d
                                              double* s) {
   double theta = pow((double)base, -2.0 * (double)i / (double)dr);
   sincos((double)p * theta, s, c);
+}
+
+// Programmatic dependent launch: every kernel of the library is launched so that it may start
+// while the previous kernel on the stream is still finishing, and waits here, after its own
+// set-up and before it touches global memory, until that kernel has completed and its writes
+// are visible. Launched without the attribute, the wait returns at once.
+__device__ __forceinline__ void wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ---- launchers (defined in the .cu files; return cudaGetLastError()) ----

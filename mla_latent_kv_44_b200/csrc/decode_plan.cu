@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p) {
   __shared__ int s_carry_a, s_carry_b;
   const int tid = threadIdx.x;
   const int64_t cap = (int64_t)p.max_blocks * p.bs;
+  wait_prior_grid();
 
   // Pass 1: attended lengths, chunk counts, exclusive prefix of chunk counts.
   if (tid == 0) s_carry_a = 0;
@@ -150,8 +151,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p) {
 }
 
 cudaError_t launch_plan(const DecodeParams& p, cudaStream_t st) {
-  plan_kernel<<<1, kPlanThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, p);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(kCombineHeads * 32) combine_kernel(DecodeParam
   __shared__ int s_slot[kRanges];
   __shared__ float s_w[kCombineHeads][kRanges];
   const int bt = blockIdx.x;
+  wait_prior_grid();
   const int nseg = p.bt_nseg[bt];
   if (nseg == 1) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -210,8 +211,7 @@ __global__ void __launch_bounds__(kCombineHeads * 32) combine_kernel(DecodeParam
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t st) {
   dim3 grid(p.BT, (p.H + kCombineHeads - 1) / kCombineHeads);
-  combine_kernel<<<grid, 128, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, grid, dim3(128), 0, st, p);
 }
 
 }  // namespace mla

@@ -19,6 +19,7 @@ template <typename T, int RW>  // RW: latent columns per lane (r <= 32 * RW)
 __global__ void __launch_bounds__(kSimtHeads * 32)
 attend_simt_kernel(DecodeParams p) {
   const int seg_id = blockIdx.x;
+  wait_prior_grid();
   if (seg_id >= p.header[0]) return;
   const Segment sg = p.segments[seg_id];
   const int bt = sg.bt, b = bt / p.T;
@@ -139,8 +140,7 @@ static cudaError_t simt_go(const DecodeParams& p, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(kRanges + p.BT, (p.H + kSimtHeads - 1) / kSimtHeads);
-  k<<<grid, kSimtHeads * 32, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, dim3(kSimtHeads * 32), smem, st, p);
 }
 
 template <typename T>

@@ -65,7 +65,10 @@ constexpr int kHdrSlots = 2;
 constexpr int kV_V = 0;
 constexpr int kV_P = kV_V + kVStages * kVStageBytes;          // 96 KB
 constexpr int kV_Hdr = kV_P + kPSlots * kPBlockBytes;         // 192 KB
-constexpr int kV_End = kV_Hdr + kHdrSlots * kHdrBytes;
+// output staging: per epilogue warp one 4 KB box of 32 rows x 32 fp32 (a TMA store source)
+constexpr int kOutBoxBytes = 32 * 32 * 4;
+constexpr int kV_Out = kV_Hdr + kHdrSlots * kHdrBytes;        // 194 KB (1 KB aligned)
+constexpr int kV_End = kV_Out + 4 * kOutBoxBytes;
 constexpr int kDataBytes = kS_End > kV_End ? kS_End : kV_End;
 
 enum Bar {
@@ -191,7 +194,9 @@ __device__ __forceinline__ int tile_block(const DecodeParams& p, const Tile& tl,
 
 __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(168)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
-                 const __grid_constant__ CUtensorMap tm_q, const DecodeParams p) {
+                 const __grid_constant__ CUtensorMap tm_q,
+                 const __grid_constant__ CUtensorMap tm_out,
+                 const __grid_constant__ CUtensorMap tm_part, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t s_base = saddr(smem);
@@ -255,6 +260,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
   tc_after();
   cluster_sync();  // barriers of both CTAs initialised before any remote traffic
   const uint32_t tmem = *tmem_slot;
+  wait_prior_grid();  // the schedule, Q and the cache rows come from earlier kernels
 
   const int q = blockIdx.x >> 1;
   int sb = 0, se = 0;
@@ -359,14 +365,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
     auto load_qckv = [&](int bt) {  // this warp's half of Q's latent part into TMEM
       const uint4* src = (const uint4*)(Q + ((size_t)bt * kH + h) * kD);
 #pragma unroll 1
-      for (int ch = 4 * half; ch < 4 * half + 4; ++ch) {
-        uint32_t w[32];
+      for (int ch = 4 * half; ch < 4 * half + 4; ch += 2) {  // 512 bytes of the row in flight
+        uint4 x[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = src[8 * ch + i];
-          w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        for (int i = 0; i < 16; ++i) x[i] = src[8 * ch + i];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            w[4 * i] = x[8 * c + i].x; w[4 * i + 1] = x[8 * c + i].y;
+            w[4 * i + 2] = x[8 * c + i].z; w[4 * i + 3] = x[8 * c + i].w;
+          }
+          tmem_st32(tq + 256 + 32 * (ch + c), w);
         }
-        tmem_st32(tq + 256 + 32 * ch, w);
       }
       tmem_wait_st();
       tc_before();
@@ -384,16 +396,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
       }
       if (!warp_wait(bar(kSFull), t & 1, ctl)) break;
       tc_after();
-      uint32_t v[128];
-      tmem_ld128(tq + 128 * half, v);
-      tc_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kSFree));  // the next tile's S may be computed now
       if (tl.last) {  // the segment's last S product is done: bring in the next query
         TileWalk look = walk;
         Tile nx;
         if (look.next(nx)) load_qckv(nx.bt);
       }
+      uint32_t v[128];
+      tmem_ld128(tq + 128 * half, v);
+      tc_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kSFree));  // the next tile's S may be computed now
       // pass 1: row max over the valid rows of both halves
       const int lim = tl.ntok - 128 * half;
       float mt = -INFINITY;
@@ -637,20 +649,36 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
         if (!wait_pv(t)) break;
         tc_after();
         const float inv_l = 1.f / l_last;
-        float* dst = tl.slot < 0 ? p.out + ((size_t)tl.bt * kH + h) * kR
-                                 : p.part_o + ((size_t)tl.slot * kH + h) * kR;
+        // O / l leaves through shared memory: each warp stages its 32 rows x 32 columns as a
+        // 128-byte-swizzled 4 KB box and one lane stores the box with TMA, so the global
+        // writes are whole lines rather than 16-byte pieces 2 KB apart.
+        const CUtensorMap* map = tl.slot < 0 ? &tm_out : &tm_part;
+        const int row0 = (tl.slot < 0 ? tl.bt : tl.slot) * kH + quad * 32;
+        const uint32_t box = s_base + kV_Out + (uint32_t)quad * kOutBoxBytes;
 #pragma unroll 1
         for (int ch = 0; ch < 16; ++ch) {
+          if (ch >= 1) {  // the previous chunk's store is done reading the box
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+          }
           uint32_t o[32];
           tmem_ld32(tq + 32 * ch, o);
-          float4* d4 = (float4*)(dst + 32 * ch);
+          const uint32_t row = box + (uint32_t)lane * 128;
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l,
-                                __uint_as_float(o[4 * i + 1]) * inv_l,
-                                __uint_as_float(o[4 * i + 2]) * inv_l,
-                                __uint_as_float(o[4 * i + 3]) * inv_l);
+          for (int u = 0; u < 8; ++u)
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             row + 16u * (uint32_t)(u ^ (lane & 7))),
+                         "f"(__uint_as_float(o[4 * u]) * inv_l),
+                         "f"(__uint_as_float(o[4 * u + 1]) * inv_l),
+                         "f"(__uint_as_float(o[4 * u + 2]) * inv_l),
+                         "f"(__uint_as_float(o[4 * u + 3]) * inv_l)
+                         : "memory");
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) tma_store(map, box, 32 * ch, row0);
         }
+        if (lane == 0) bulk_wait_read<0>();  // the box is free for the next segment
+        __syncwarp();
         tc_before();
       }
       ++t;
@@ -658,6 +686,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
   }
 
   // ---------------------------------------------------------------------- teardown
+  if (!score && warp >= 2 && warp < 6 && lane == 0) bulk_wait_all();  // output stores landed
   tc_before();
   __syncthreads();
   tc_after();
@@ -680,9 +709,11 @@ bool tc_supported(const mla_config& c) {
 
 cudaError_t launch_attend_tc(const mla_config& c, const DecodeParams& p, cudaStream_t st) {
   (void)c;
-  CUtensorMap kv, qm;
+  CUtensorMap kv, qm, om, pm;
   if (!make_bf16_map(&kv, p.pool, kD, (uint64_t)p.num_blocks * kRows, kD * 2, kRows) ||
-      !make_bf16_map(&qm, p.q, kD, (uint64_t)p.BT * kH, kD * 2, kH))
+      !make_bf16_map(&qm, p.q, kD, (uint64_t)p.BT * kH, kD * 2, kH) ||
+      !make_f32_box32_map(&om, p.out, kR, (uint64_t)p.BT * kH) ||
+      !make_f32_box32_map(&pm, p.part_o, kR, (uint64_t)kMaxPartials * kH))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
@@ -691,8 +722,8 @@ cudaError_t launch_attend_tc(const mla_config& c, const DecodeParams& p, cudaStr
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  attend_tc_kernel<<<2 * kRanges, kThreads, kSmemBytes, st>>>(kv, qm, p);
-  return cudaGetLastError();
+  return launch_pdl(attend_tc_kernel, dim3(2 * kRanges), dim3(kThreads), kSmemBytes, st, kv, qm,
+                    om, pm, p);
 }
 
 }  // namespace mla

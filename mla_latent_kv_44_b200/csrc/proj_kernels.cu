@@ -21,6 +21,7 @@ absorb_kernel(const T* __restrict__ q_nope, const T* __restrict__ q_rope,
               const int32_t* __restrict__ pos, const T* __restrict__ w_uk, T* __restrict__ q_out,
               int n, int H, int dh, int r, int dr, float base) {
   extern __shared__ float s_q[];  // kAbsorbTokens x dh
+  wait_prior_grid();
   const int h = blockIdx.y;
   const int n0 = blockIdx.x * kAbsorbTokens;
   const int nt = min(kAbsorbTokens, n - n0);
@@ -86,9 +87,8 @@ static cudaError_t absorb_go(const mla_config& c, const void* qn, const void* qr
     if (e != cudaSuccess) return e;
   }
   dim3 grid((n + kAbsorbTokens - 1) / kAbsorbTokens, c.num_heads);
-  k<<<grid, 256, smem, st>>>((const T*)qn, (const T*)qr, pos, (const T*)w, (T*)q, n, c.num_heads,
-                             c.head_dim, c.kv_rank, c.rope_dim, c.rope_base);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, dim3(256), smem, st, (const T*)qn, (const T*)qr, pos, (const T*)w,
+                    (T*)q, n, c.num_heads, c.head_dim, c.kv_rank, c.rope_dim, c.rope_base);
 }
 
 template <typename T>
@@ -121,6 +121,7 @@ append_kernel(const T* __restrict__ ckv, const T* __restrict__ kr, const float* 
               uint32_t* err) {
   const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
+  wait_prior_grid();
   if (row >= n) return;
   const int b = seq[row], p = pos[row];
   if (b < 0 || b >= batch || p < 0 || (int64_t)p >= (int64_t)max_blocks * bs) {
@@ -159,16 +160,14 @@ cudaError_t launch_append(const mla_config& c, const void* ckv, const void* kr,
   const int threads = 256, rows_per_cta = threads / 32;
   const int grid = (n + rows_per_cta - 1) / rows_per_cta;
   if (c.dtype == MLA_BF16)
-    append_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
-        (const __nv_bfloat16*)ckv, (const __nv_bfloat16*)kr, gamma, seq, pos, table, batch,
-        max_blocks, (__nv_bfloat16*)pool, num_blocks, n, c.kv_rank, c.rope_dim, c.block_size,
-        c.rms_eps, c.rope_base, err);
-  else
-    append_kernel<float><<<grid, threads, 0, st>>>(
-        (const float*)ckv, (const float*)kr, gamma, seq, pos, table, batch, max_blocks,
-        (float*)pool, num_blocks, n, c.kv_rank, c.rope_dim, c.block_size, c.rms_eps,
-        c.rope_base, err);
-  return cudaGetLastError();
+    return launch_pdl(append_kernel<__nv_bfloat16>, dim3(grid), dim3(threads), 0, st,
+                      (const __nv_bfloat16*)ckv, (const __nv_bfloat16*)kr, gamma, seq, pos, table,
+                      batch, max_blocks, (__nv_bfloat16*)pool, num_blocks, n, c.kv_rank,
+                      c.rope_dim, c.block_size, c.rms_eps, c.rope_base, err);
+  return launch_pdl(append_kernel<float>, dim3(grid), dim3(threads), 0, st, (const float*)ckv,
+                    (const float*)kr, gamma, seq, pos, table, batch, max_blocks, (float*)pool,
+                    num_blocks, n, c.kv_rank, c.rope_dim, c.block_size, c.rms_eps, c.rope_base,
+                    err);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -182,6 +181,7 @@ __global__ void __launch_bounds__(256)
 output_kernel(const float* __restrict__ lat, const T* __restrict__ w_uv, T* __restrict__ o, int n,
               int H, int dv, int r) {
   extern __shared__ float s_lat[];  // kOutTokens x r
+  wait_prior_grid();
   const int h = blockIdx.y;
   const int n0 = blockIdx.x * kOutTokens;
   const int nt = min(kOutTokens, n - n0);
@@ -217,16 +217,15 @@ cudaError_t launch_output(const mla_config& c, const float* lat, const void* w_u
     auto k = output_kernel<__nv_bfloat16>;
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, 256, smem, st>>>(lat, (const __nv_bfloat16*)w_uv, (__nv_bfloat16*)o, n,
-                               c.num_heads, c.head_dim_v, c.kv_rank);
+    return launch_pdl(k, grid, dim3(256), smem, st, lat, (const __nv_bfloat16*)w_uv,
+                      (__nv_bfloat16*)o, n, c.num_heads, c.head_dim_v, c.kv_rank);
   } else {
     auto k = output_kernel<float>;
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, 256, smem, st>>>(lat, (const float*)w_uv, (float*)o, n, c.num_heads,
-                               c.head_dim_v, c.kv_rank);
+    return launch_pdl(k, grid, dim3(256), smem, st, lat, (const float*)w_uv, (float*)o, n,
+                      c.num_heads, c.head_dim_v, c.kv_rank);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace mla

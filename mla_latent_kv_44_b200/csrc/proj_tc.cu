@@ -113,6 +113,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
   __syncthreads();
   tc_after();
   const uint32_t tmem = *tmem_slot;
+  wait_prior_grid();
 
   bool ok = true;
   if (threadIdx.x == 0) {
@@ -238,6 +239,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const OutputArgs a) {
   __syncthreads();
   tc_after();
   const uint32_t tmem = *tmem_slot;
+  wait_prior_grid();
 
   bool ok = true;
   for (int c = 0; c < nchunks && ok; ++c) {
@@ -390,8 +392,7 @@ cudaError_t launch_absorb_tc(const mla_config& c, const void* q_nope, const void
   AbsorbArgs a{(const __nv_bfloat16*)q_rope, pos, (__nv_bfloat16*)q_out, err, n, H, dh, r,
                c.rope_dim, tile, c.rope_base};
   dim3 grid((n + tile - 1) / tile, jts, H);
-  absorb_tc_kernel<<<grid, 128, smem, st>>>(tw, tq, a);
-  return cudaGetLastError();
+  return launch_pdl(absorb_tc_kernel, grid, dim3(128), smem, st, tw, tq, a);
 }
 
 cudaError_t launch_output_tc(const mla_config& c, const float* lat, const void* w_uv, void* o,
@@ -409,8 +410,7 @@ cudaError_t launch_output_tc(const mla_config& c, const float* lat, const void* 
   if (e != cudaSuccess) return e;
   OutputArgs a{lat, (__nv_bfloat16*)o, err, n, H, dv, r, tile};
   dim3 grid((n + tile - 1) / tile, mts, H);
-  output_tc_kernel<<<grid, 256, smem, st>>>(tw, a);
-  return cudaGetLastError();
+  return launch_pdl(output_tc_kernel, grid, dim3(256), smem, st, tw, a);
 }
 
 }  // namespace mla
