@@ -380,33 +380,74 @@ def run_ours(args, w):
     stage_ms = {n: sum(evd[k][i].elapsed_time(evd[k][i + 1]) for k in range(n_detail)) / n_detail
                 for i, n in enumerate(names)}
 
-    # ---- e2e through host buffers: H2D of the step's inputs, the four calls, D2H of o ----
-    host_in = [t.cpu().pin_memory() for t in (st.q_nope, st.q_rope, st.ckv_new, st.krope_new,
-                                              st.seq_new, st.pos_new, st.seq_lens)]
-    dev_in = [st.q_nope, st.q_rope, st.ckv_new, st.krope_new, st.seq_new, st.pos_new, st.seq_lens]
-    host_out = torch.empty(st.o.shape, dtype=st.o.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = host_out.numel() * host_out.element_size()
+    # ---- e2e through host buffers: every step uploads its inputs from pinned host memory (one
+    # packed copy) and reads its output o back. Steps are pipelined over two input and two
+    # output buffer sets: step k+1's upload and step k-1's download run on copy streams while
+    # step k computes.
+    fields = ["q_nope", "q_rope", "ckv_new", "krope_new", "seq_new", "pos_new", "seq_lens"]
+    layout, total = [], 0
+    for f in fields:
+        t_ = getattr(st, f)
+        nbytes = t_.numel() * t_.element_size()
+        layout.append((f, total, nbytes, t_.dtype, tuple(t_.shape)))
+        total = (total + nbytes + 255) // 256 * 256
+    host_in = torch.empty(total, dtype=torch.uint8).pin_memory()
+    for f, off, nbytes, _, _ in layout:
+        host_in[off:off + nbytes].copy_(getattr(st, f).contiguous().view(-1).view(torch.uint8).cpu())
+    dev_sets = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
+    views = [{f: dev_sets[i][off:off + nbytes].view(dt).view(shape)
+              for f, off, nbytes, dt, shape in layout} for i in range(2)]
+    outs = [torch.empty_like(st.o) for _ in range(2)]
+    host_out = [torch.empty(st.o.shape, dtype=st.o.dtype).pin_memory() for _ in range(2)]
+    h2d = total
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    mk = lambda: [torch.cuda.Event() for _ in range(2)]
+    ev_in, ev_used, ev_done, ev_read = mk(), mk(), mk(), mk()
+
+    def upload(k):
+        i = k % 2
+        with torch.cuda.stream(up):
+            if k >= 2:
+                up.wait_event(ev_used[i])         # step k-2 finished reading this set
+            dev_sets[i].copy_(host_in, non_blocking=True)
+            ev_in[i].record(up)
+
+    def run_e2e(n):
+        upload(0)
+        for k in range(n):
+            i = k % 2
+            if k + 1 < n:
+                upload(k + 1)
+            stream.wait_event(ev_in[i])
+            if k >= 2:
+                stream.wait_event(ev_read[i])     # step k-2's output has been read back
+            for f in fields:
+                setattr(st, f, views[i][f])
+            st.o = outs[i]
+            st.step(stream)
+            ev_used[i].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_used[i])
+                host_out[i].copy_(outs[i], non_blocking=True)
+                ev_read[i].record(down)
+        last = [ev_read[(n - 1) % 2]] + ([ev_read[n % 2]] if n > 1 else [])
+        for e_ in last:
+            stream.wait_event(e_)
+
     e2e_steps = min(args.steps, 200)
     with torch.cuda.stream(stream):
-        for _ in range(3):
-            for hsrc, ddst in zip(host_in, dev_in):
-                ddst.copy_(hsrc, non_blocking=True)
-            st.step(stream)
-            host_out.copy_(st.o, non_blocking=True)
-    stream.synchronize()
+        run_e2e(3)
+    torch.cuda.synchronize(dev)
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for _ in range(e2e_steps):
-            for hsrc, ddst in zip(host_in, dev_in):
-                ddst.copy_(hsrc, non_blocking=True)
-            st.step(stream)
-            host_out.copy_(st.o, non_blocking=True)
+        up.wait_event(e0)
+        run_e2e(e2e_steps)
         e1.record(stream)
-    stream.synchronize()
+    torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
     barrier()
 

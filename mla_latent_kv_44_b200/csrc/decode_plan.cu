@@ -193,18 +193,31 @@ __global__ void __launch_bounds__(kCombineHeads * 32) combine_kernel(DecodeParam
   for (int k = lane; k < nseg; k += 32)
     s_w[warp][k] = expf(p.part_lse[(size_t)s_slot[k] * p.H + h] - L);
   __syncwarp();
-  for (int d = lane; d < r4; d += 32) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
+  // a lane holds up to four float4 of the row at once (r = 512 in one pass), so every partial's
+  // loads for the whole row are in flight together
+  for (int d0 = lane; d0 < r4; d0 += 128) {
+    float4 acc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
     for (int k = 0; k < nseg; ++k) {
       const float w = s_w[warp][k];
-      const float4 v = __ldcs((const float4*)(p.part_o + ((size_t)s_slot[k] * p.H + h) * p.r) + d);
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
+      const float4* src = (const float4*)(p.part_o + ((size_t)s_slot[k] * p.H + h) * p.r);
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        v[u] = (d0 + 32 * u < r4) ? __ldcs(src + d0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc[u].x = fmaf(w, v[u].x, acc[u].x);
+        acc[u].y = fmaf(w, v[u].y, acc[u].y);
+        acc[u].z = fmaf(w, v[u].z, acc[u].z);
+        acc[u].w = fmaf(w, v[u].w, acc[u].w);
+      }
     }
-    dst[d] = acc;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (d0 + 32 * u < r4) dst[d0 + 32 * u] = acc[u];
   }
   if (lane == 0 && p.lse) p.lse[(size_t)bt * p.H + h] = L;
 }

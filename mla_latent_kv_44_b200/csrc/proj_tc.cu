@@ -28,6 +28,8 @@ constexpr int kWRows = 128;        // weight rows per CTA = MMA M
 constexpr int kMaxTokTile = 128;   // tokens per CTA at most = MMA N (TMEM columns)
 constexpr uint32_t kProjTmemCols = 128;
 constexpr int kSlab = 64;          // bf16 elements per 128-byte swizzled row
+constexpr int kOutTokTile = 64;    // tokens per CTA of the output kernel at most
+constexpr int kOutItems = kOutTokTile * 16 / 256;  // 8-float groups per thread and chunk
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint32_t* err) {
   if (mbar_try(bar, parity)) return true;
@@ -125,20 +127,28 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
   }
 
   // RoPE part of the query, while the copies are in flight: pairs (2i, 2i+1) rotated by
-  // pos * base^(-2i/d_r), angle in double; the (token, pair) items of this head are dealt out
-  // over its gridDim.y CTAs
+  // pos * base^(-2i/d_r), angle and rotation in double. The angles depend on the token only, so
+  // each token of this tile is given to one CTA of the tile (CTA (jt, h) takes the tokens
+  // t = jt + gridDim.y * h, ...), which takes the d_r/2 sin/cos pairs once into shared memory
+  // and rotates the token's query in every head.
   const int D = a.r + a.dr;
   const int half = a.dr / 2;
-  for (int idx = jt * blockDim.x + threadIdx.x; idx < ntok * half; idx += gridDim.y * blockDim.x) {
-    const int t = idx / half, i = idx - t * half;
+  double* cs_tab = (double*)(ctl + 64);  // [2][half] cos, sin
+  for (int t = jt + gridDim.y * h; t < ntok; t += gridDim.y * gridDim.z) {
     const int n = n0 + t;
-    double cs, sn;
-    rope_cos_sin(a.pos[n], i, a.dr, a.base, &cs, &sn);
-    const __nv_bfloat16* src = a.q_rope + ((size_t)n * a.H + h) * a.dr;
-    const double x0 = __bfloat162float(src[2 * i]), x1 = __bfloat162float(src[2 * i + 1]);
-    __nv_bfloat16* dst = a.q_out + ((size_t)n * a.H + h) * D + a.r;
-    dst[2 * i] = __float2bfloat16_rn((float)(x0 * cs - x1 * sn));
-    dst[2 * i + 1] = __float2bfloat16_rn((float)(x0 * sn + x1 * cs));
+    __syncthreads();  // the previous token's table is no longer read
+    for (int i = threadIdx.x; i < half; i += blockDim.x)
+      rope_cos_sin(a.pos[n], i, a.dr, a.base, &cs_tab[i], &cs_tab[half + i]);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < a.H * half; idx += blockDim.x) {
+      const int hh = idx / half, i = idx - hh * half;
+      const double cs = cs_tab[i], sn = cs_tab[half + i];
+      const __nv_bfloat16* src = a.q_rope + ((size_t)n * a.H + hh) * a.dr;
+      const double x0 = __bfloat162float(src[2 * i]), x1 = __bfloat162float(src[2 * i + 1]);
+      __nv_bfloat16* dst = a.q_out + ((size_t)n * a.H + hh) * D + a.r;
+      dst[2 * i] = __float2bfloat16_rn((float)(x0 * cs - x1 * sn));
+      dst[2 * i + 1] = __float2bfloat16_rn((float)(x0 * sn + x1 * cs));
+    }
   }
 
   if (threadIdx.x == 0) {
@@ -241,6 +251,40 @@ output_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const OutputArgs a) {
   const uint32_t tmem = *tmem_slot;
   wait_prior_grid();
 
+  // The weights of chunk c go by TMA into stage c & 1 as soon as that stage is free (chunks 0
+  // and 1 at once). The latent of chunk c + 1 is loaded into registers while chunk c's MMAs
+  // run: each thread holds kOutItems groups of 8 floats (tile <= 64 tokens x 16 groups).
+  auto issue_w = [&](int c) {
+    const int s = c & 1;
+    const int k0 = c * 128, nsl = min(128, a.r - k0) / kSlab;
+    mbar_expect_tx(bar_full + 8 * s, nsl * kSlabA);
+    for (int k = 0; k < nsl; ++k)
+      tma_load(s0 + s * stage_bytes + k * kSlabA, &tm_w, bar_full + 8 * s, k0 + kSlab * k,
+               h * a.dv + i0);
+    flags[1] = c + 1;
+  };
+  float4 pf[2 * kOutItems];
+  auto load_lat = [&](int c) {
+    const int k0 = c * 128, groups = min(128, a.r - k0) / 8;
+#pragma unroll
+    for (int it = 0; it < kOutItems; ++it) {
+      const int idx = threadIdx.x + it * blockDim.x;
+      const int t = idx / groups, q = idx - t * groups;
+      pf[2 * it] = pf[2 * it + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < ntok) {
+        const float4* src =
+            (const float4*)(a.lat + ((size_t)(n0 + t) * a.H + h) * a.r + k0 + 8 * q);
+        pf[2 * it] = __ldg(src);
+        pf[2 * it + 1] = __ldg(src + 1);
+      }
+    }
+  };
+  if (threadIdx.x == 0) {
+    issue_w(0);
+    if (nchunks > 1) issue_w(1);
+  }
+  load_lat(0);
+
   bool ok = true;
   for (int c = 0; c < nchunks && ok; ++c) {
     const int s = c & 1;
@@ -248,42 +292,35 @@ output_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const OutputArgs a) {
     uint8_t* pB = smem + s * stage_bytes + 2 * kSlabA;
     const int k0 = c * 128;
     const int width = min(128, a.r - k0);   // 64 or 128 (r is a multiple of 64)
-    const int nsl = width / kSlab;
     if (c >= 2) {  // stage s is free once the MMAs of chunk c - 2 are done
       ok = __syncthreads_and(wait_bounded(bar_done + 8 * s, ((c - 2) >> 1) & 1, a.err));
       if (!ok) break;
-    }
-    if (threadIdx.x == 0) {
-      mbar_expect_tx(bar_full + 8 * s, nsl * kSlabA);
-      for (int k = 0; k < nsl; ++k)
-        tma_load(sA + k * kSlabA, &tm_w, bar_full + 8 * s, k0 + kSlab * k, h * a.dv + i0);
-      flags[1] = c + 1;
+      if (threadIdx.x == 0) issue_w(c);
     }
     // o_lat chunk -> hi and lo bf16 terms, swizzled K-major: row t, 16-byte group g of slab
     // k at g ^ (t & 7); the lo slabs follow the two hi slabs
     const int groups = width / 8;
-    for (int idx = threadIdx.x; idx < a.tile * groups; idx += blockDim.x) {
-      const int t = idx / groups, q = idx - t * groups;
-      const int k = q >> 3, g = q & 7;
-      float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (t < ntok) {
-        const float4* src =
-            (const float4*)(a.lat + ((size_t)(n0 + t) * a.H + h) * a.r + k0 + 8 * q);
-        const float4 u = __ldg(src), v = __ldg(src + 1);
-        x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
-        x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
-      }
-      uint32_t hi[4], lo[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
-        hi[e] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
-        lo[e] = pack_bf16(x[2 * e] - __bfloat162float(h0), x[2 * e + 1] - __bfloat162float(h1));
+    for (int it = 0; it < kOutItems; ++it) {
+      const int idx = threadIdx.x + it * blockDim.x;
+      const int t = idx / groups, q = idx - t * groups;
+      if (t < a.tile) {
+        const int k = q >> 3, g = q & 7;
+        const float x[8] = {pf[2 * it].x, pf[2 * it].y, pf[2 * it].z, pf[2 * it].w,
+                            pf[2 * it + 1].x, pf[2 * it + 1].y, pf[2 * it + 1].z, pf[2 * it + 1].w};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
+          hi[e] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+          lo[e] = pack_bf16(x[2 * e] - __bfloat162float(h0), x[2 * e + 1] - __bfloat162float(h1));
+        }
+        const uint32_t off = k * slab_b + t * 128 + ((g ^ (t & 7)) << 4);
+        *(uint4*)(pB + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *(uint4*)(pB + 2 * slab_b + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
-      const uint32_t off = k * slab_b + t * 128 + ((g ^ (t & 7)) << 4);
-      *(uint4*)(pB + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *(uint4*)(pB + 2 * slab_b + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
+    if (c + 1 < nchunks) load_lat(c + 1);  // in flight during this chunk's MMAs
     fence_proxy_async();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -344,18 +381,20 @@ output_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const OutputArgs a) {
 }
 
 // Tokens per CTA: enough token tiles that the grid covers the 148 SMs about twice, each a
-// multiple of 16 (the MMA's N step) and at most 128 (the TMEM accumulator's columns).
-int token_tile(int n, int ctas_per_tile) {
+// multiple of 16 (the MMA's N step) and at most max_tile (128, the TMEM accumulator's columns,
+// for the query; 64 for the output, whose threads hold a chunk of the latent in registers).
+int token_tile(int n, int ctas_per_tile, int max_tile) {
   const int want = (2 * 148 + ctas_per_tile - 1) / ctas_per_tile;
-  int tiles = (n + kMaxTokTile - 1) / kMaxTokTile;
+  int tiles = (n + max_tile - 1) / max_tile;
   tiles = std::max(tiles, std::min(want, (n + 15) / 16));
-  return std::min(kMaxTokTile, round_up((n + tiles - 1) / tiles, 16));
+  return std::min(max_tile, round_up((n + tiles - 1) / tiles, 16));
 }
 
-size_t absorb_smem(int dh, int tile) {
-  const size_t need = 1024 + 2 * (size_t)dh * 128 + (size_t)(dh / kSlab) * round_up(tile * 128, 1024) + 64;
-  // at least 61 KB: no more than three CTAs (3 x 128 TMEM columns) share an SM
-  return std::max(need, (size_t)61 * 1024);
+size_t absorb_smem(int dh, int dr, int tile) {
+  const size_t need = 1024 + 2 * (size_t)dh * 128 +
+                      (size_t)(dh / kSlab) * round_up(tile * 128, 1024) + 64 + 8 * (size_t)dr;
+  // at least 51 KB: no more than four CTAs (4 x 128 TMEM columns) share an SM
+  return std::max(need, (size_t)51 * 1024);
 }
 
 size_t output_smem(int tile) {
@@ -379,13 +418,13 @@ cudaError_t launch_absorb_tc(const mla_config& c, const void* q_nope, const void
                              uint32_t* err, cudaStream_t st) {
   const int H = c.num_heads, dh = c.head_dim, r = c.kv_rank;
   const int jts = (r + kWRows - 1) / kWRows;
-  const int tile = token_tile(n, jts * H);
+  const int tile = token_tile(n, jts * H, kMaxTokTile);
   CUtensorMap tw, tq;
   if (!make_bf16_map(&tw, w_uk, (uint64_t)r, (uint64_t)H * dh, (uint64_t)r * 2, (uint32_t)dh) ||
       !make_bf16_map(&tq, q_nope, (uint64_t)H * dh, (uint64_t)n, (uint64_t)H * dh * 2,
                      (uint32_t)tile))
     return cudaErrorInvalidValue;
-  const size_t smem = absorb_smem(dh, tile);
+  const size_t smem = absorb_smem(dh, c.rope_dim, tile);
   cudaError_t e = cudaFuncSetAttribute(absorb_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -399,7 +438,7 @@ cudaError_t launch_output_tc(const mla_config& c, const float* lat, const void* 
                              int n, uint32_t* err, cudaStream_t st) {
   const int H = c.num_heads, dv = c.head_dim_v, r = c.kv_rank;
   const int mts = (dv + kWRows - 1) / kWRows;
-  const int tile = token_tile(n, mts * H);
+  const int tile = token_tile(n, mts * H, kOutTokTile);
   if (((uintptr_t)lat & 15) != 0) return cudaErrorInvalidValue;
   CUtensorMap tw;
   if (!make_bf16_map(&tw, w_uv, (uint64_t)r, (uint64_t)H * dv, (uint64_t)r * 2, kWRows))
