@@ -93,8 +93,10 @@ typedef struct {
  * pos (n_tokens) int32 >= 0; w_uk (H, d_h, r) dtype -- the nn.Linear(r, H*d_h) weight,
  * rows h*d_h .. (h+1)*d_h-1 for head h, i.e. the same memory without a transpose;
  * q_out (n_tokens, H, r + d_r) dtype, rounded to nearest even when bf16.
- * dev_err may be NULL; the tensor-core kernel sets MLA_DEV_WAIT_TIMEOUT in it when one of its
- * bounded waits gives up (that tile of q_out is then not written).
+ * The tensor-core kernel (bf16, d_h a multiple of 64 up to 256, r a multiple of 64, d_r a
+ * multiple of 8, every pointer 16-byte aligned) is used where it applies. dev_err may be NULL;
+ * that kernel sets MLA_DEV_WAIT_TIMEOUT in it when one of its bounded waits gives up (that
+ * tile of q_out is then not written).
  */
 MLA_API mla_status mla_absorb_query(const mla_config* cfg, const void* q_nope, const void* q_rope,
                             const int32_t* pos, const void* w_uk, void* q_out, int32_t n_tokens,

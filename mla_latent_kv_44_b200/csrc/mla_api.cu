@@ -56,7 +56,8 @@ mla_status mla_absorb_query(const mla_config* cfg, const void* q_nope, const voi
     return MLA_ERR_INVALID_ARG;
   if (n_tokens > (1 << 24)) return MLA_ERR_UNSUPPORTED;
   const bool tc = cfg->decode_kernel != MLA_DECODE_SIMT && absorb_tc_supported(*cfg) &&
-                  aligned(q_nope, 16) && aligned(w_uk, 16);
+                  aligned(q_nope, 16) && aligned(w_uk, 16) && aligned(q_out, 16) &&
+                  (cfg->rope_dim == 0 || aligned(q_rope, 16));
   if (cfg->decode_kernel == MLA_DECODE_TENSOR && !tc) return MLA_ERR_UNSUPPORTED;
   if (tc)
     return from_cuda(launch_absorb_tc(*cfg, q_nope, q_rope, pos, w_uk, q_out, n_tokens, dev_err,

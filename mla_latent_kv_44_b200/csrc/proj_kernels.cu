@@ -118,7 +118,7 @@ append_kernel(const T* __restrict__ ckv, const T* __restrict__ kr, const float* 
               const int32_t* __restrict__ seq, const int32_t* __restrict__ pos,
               const int32_t* __restrict__ table, int batch, int max_blocks, T* __restrict__ pool,
               int num_blocks, int n, int r, int dr, int bs, float eps, float base,
-              uint32_t* err) {
+              uint32_t* err, bool vec) {
   const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   wait_prior_grid();
@@ -134,15 +134,55 @@ append_kernel(const T* __restrict__ ckv, const T* __restrict__ kr, const float* 
     return;
   }
   const T* x = ckv + (size_t)row * r;
-  float ss = 0.f;
-  for (int j = lane; j < r; j += 32) {
-    const float v = to_f32(x[j]);
-    ss = fmaf(v, v, ss);
-  }
-  ss = warp_sum(ss);
-  const float inv = 1.0f / sqrtf(ss / (float)r + eps);
   T* dst = pool + ((size_t)blk * bs + (p % bs)) * (size_t)(r + dr);
-  for (int j = lane; j < r; j += 32) dst[j] = from_f32<T>(to_f32(x[j]) * inv * gamma[j]);
+  if (vec) {
+    // bf16 rows, r a multiple of 256, 16-byte aligned: lane l owns the r/32 contiguous values
+    // [l * r/32, (l+1) * r/32), up to four 16-byte pieces loaded together
+    const int E = r / 32, pieces = E / 8;
+    uint4 xv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k < pieces) xv[k] = ((const uint4*)(x + lane * E))[k];
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (k >= pieces) break;
+      const uint32_t w[4] = {xv[k].x, xv[k].y, xv[k].z, xv[k].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float a0 = __uint_as_float(w[u] << 16), a1 = __uint_as_float(w[u] & 0xffff0000u);
+        ss = fmaf(a0, a0, ss);
+        ss = fmaf(a1, a1, ss);
+      }
+    }
+    ss = warp_sum(ss);
+    const float inv = 1.0f / sqrtf(ss / (float)r + eps);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (k >= pieces) break;
+      const float4 g0 = ((const float4*)(gamma + lane * E))[2 * k];
+      const float4 g1 = ((const float4*)(gamma + lane * E))[2 * k + 1];
+      const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      const uint32_t w[4] = {xv[k].x, xv[k].y, xv[k].z, xv[k].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float a0 = __uint_as_float(w[u] << 16), a1 = __uint_as_float(w[u] & 0xffff0000u);
+        const __nv_bfloat162 v = __floats2bfloat162_rn(a0 * inv * gg[2 * u], a1 * inv * gg[2 * u + 1]);
+        o[u] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+      ((uint4*)(dst + lane * E))[k] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  } else {
+    float ss = 0.f;
+    for (int j = lane; j < r; j += 32) {
+      const float v = to_f32(x[j]);
+      ss = fmaf(v, v, ss);
+    }
+    ss = warp_sum(ss);
+    const float inv = 1.0f / sqrtf(ss / (float)r + eps);
+    for (int j = lane; j < r; j += 32) dst[j] = from_f32<T>(to_f32(x[j]) * inv * gamma[j]);
+  }
   const T* k = kr + (size_t)row * dr;
   for (int i = lane; i < dr / 2; i += 32) {
     double c, s;
@@ -159,15 +199,20 @@ cudaError_t launch_append(const mla_config& c, const void* ckv, const void* kr,
                           int num_blocks, int n, uint32_t* err, cudaStream_t st) {
   const int threads = 256, rows_per_cta = threads / 32;
   const int grid = (n + rows_per_cta - 1) / rows_per_cta;
-  if (c.dtype == MLA_BF16)
+  if (c.dtype == MLA_BF16) {
+    // contiguous 16-byte pieces per lane: r a multiple of 256 (at most 1024), aligned rows
+    const bool vec = c.kv_rank % 256 == 0 && c.kv_rank <= 1024 && ((uintptr_t)ckv & 15) == 0 &&
+                     ((uintptr_t)gamma & 15) == 0 && ((uintptr_t)pool & 15) == 0 &&
+                     ((c.kv_rank + c.rope_dim) * 2) % 16 == 0;
     return launch_pdl(append_kernel<__nv_bfloat16>, dim3(grid), dim3(threads), 0, st,
                       (const __nv_bfloat16*)ckv, (const __nv_bfloat16*)kr, gamma, seq, pos, table,
                       batch, max_blocks, (__nv_bfloat16*)pool, num_blocks, n, c.kv_rank,
-                      c.rope_dim, c.block_size, c.rms_eps, c.rope_base, err);
+                      c.rope_dim, c.block_size, c.rms_eps, c.rope_base, err, vec);
+  }
   return launch_pdl(append_kernel<float>, dim3(grid), dim3(threads), 0, st, (const float*)ckv,
                     (const float*)kr, gamma, seq, pos, table, batch, max_blocks, (float*)pool,
                     num_blocks, n, c.kv_rank, c.rope_dim, c.block_size, c.rms_eps, c.rope_base,
-                    err);
+                    err, false);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -29,6 +29,7 @@ constexpr int kMaxTokTile = 128;   // tokens per CTA at most = MMA N (TMEM colum
 constexpr uint32_t kProjTmemCols = 128;
 constexpr int kSlab = 64;          // bf16 elements per 128-byte swizzled row
 constexpr int kOutTokTile = 64;    // tokens per CTA of the output kernel at most
+constexpr int kRopeVec = 8;        // 16-byte pieces of q_rope a thread has in flight
 constexpr int kOutItems = kOutTokTile * 16 / 256;  // 8-float groups per thread and chunk
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint32_t* err) {
@@ -140,14 +141,33 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
     for (int i = threadIdx.x; i < half; i += blockDim.x)
       rope_cos_sin(a.pos[n], i, a.dr, a.base, &cs_tab[i], &cs_tab[half + i]);
     __syncthreads();
-    for (int idx = threadIdx.x; idx < a.H * half; idx += blockDim.x) {
-      const int hh = idx / half, i = idx - hh * half;
-      const double cs = cs_tab[i], sn = cs_tab[half + i];
-      const __nv_bfloat16* src = a.q_rope + ((size_t)n * a.H + hh) * a.dr;
-      const double x0 = __bfloat162float(src[2 * i]), x1 = __bfloat162float(src[2 * i + 1]);
-      __nv_bfloat16* dst = a.q_out + ((size_t)n * a.H + hh) * D + a.r;
-      dst[2 * i] = __float2bfloat16_rn((float)(x0 * cs - x1 * sn));
-      dst[2 * i + 1] = __float2bfloat16_rn((float)(x0 * sn + x1 * cs));
+    // the token's q_rope rows of all heads (H x d_r bf16, contiguous) in 16-byte pieces, kRopeVec
+    // pieces per thread loaded together, rotated, stored into the RoPE part of each Q row
+    const int pieces = a.H * a.dr / 8;
+    const uint4* src = (const uint4*)(a.q_rope + (size_t)n * a.H * a.dr);
+    for (int base = 0; base < pieces; base += kRopeVec * blockDim.x) {
+      uint4 x[kRopeVec];
+#pragma unroll
+      for (int k = 0; k < kRopeVec; ++k) {
+        const int pc = base + k * blockDim.x + threadIdx.x;
+        if (pc < pieces) x[k] = src[pc];
+      }
+#pragma unroll
+      for (int k = 0; k < kRopeVec; ++k) {
+        const int pc = base + k * blockDim.x + threadIdx.x;
+        if (pc >= pieces) break;
+        const int hh = pc / (a.dr / 8), e0 = (pc - hh * (a.dr / 8)) * 8;  // first of 8 values
+        const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = e0 / 2 + u;  // pair index
+          const double cs = cs_tab[i], sn = cs_tab[half + i];
+          const double x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xffff0000u);
+          o[u] = pack_bf16((float)(x0 * cs - x1 * sn), (float)(x0 * sn + x1 * cs));
+        }
+        *(uint4*)(a.q_out + ((size_t)n * a.H + hh) * D + a.r + e0) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
   }
 
@@ -406,7 +426,7 @@ size_t output_smem(int tile) {
 
 bool absorb_tc_supported(const mla_config& c) {
   return c.dtype == MLA_BF16 && c.head_dim % kSlab == 0 && c.head_dim <= 256 &&
-         c.kv_rank % kSlab == 0 && c.rope_dim % 2 == 0;
+         c.kv_rank % kSlab == 0 && c.rope_dim % 8 == 0;
 }
 
 bool output_tc_supported(const mla_config& c) {

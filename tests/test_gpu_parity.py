@@ -112,6 +112,7 @@ _SIMT, _TC = 1, 2  # mla_config.decode_kernel: CUDA-core or tensor-core kernels
     ("bf16", (128, 128, 512, 64), 64, _TC),
     ("bf16", (128, 128, 512, 64), 200, _TC),
     ("bf16", (4, 256, 192, 0), 300, _TC),
+    ("bf16", (8, 64, 128, 8), 5, _TC),
 ])
 def test_absorb_stage(mla, dtype, shape, N, kernel):
     H, dh, r, dr = shape
@@ -148,7 +149,8 @@ def test_absorb_stage(mla, dtype, shape, N, kernel):
 # Stage: append (integer placement bit-exact, values within one rounding)
 # ----------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("dtype,r,dr", [("f32", 64, 16), ("bf16", 64, 32), ("bf16", 512, 64)])
+@pytest.mark.parametrize("dtype,r,dr", [("f32", 64, 16), ("bf16", 64, 32), ("bf16", 512, 64),
+                                       ("bf16", 1024, 0), ("bf16", 256, 8)])
 def test_append_stage(mla, dtype, r, dr):
     g = np.random.default_rng([1, 2])
     B, maxb, bs, nb = 3, 4, 16, 14
