@@ -70,7 +70,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p) {
   const int64_t cap = (int64_t)p.max_blocks * p.bs;
   wait_prior_grid();
 
-  // Pass 1: attended lengths, chunk counts, exclusive prefix of chunk counts.
+  // Pass 1: attended lengths, chunk counts, exclusive prefix of chunk counts. With at most
+  // kPlanThreads row groups (one pass), pass 2 takes them from registers.
+  int my_len = 0, my_chunk0 = 0;
   if (tid == 0) s_carry_a = 0;
   __syncthreads();
   for (int base = 0; base < p.BT; base += kPlanThreads) {
@@ -87,10 +89,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p) {
       }
       nch = (len + kChunk - 1) / kChunk;
       p.bt_len[bt] = len;
+      my_len = len;
     }
     int inc = nch, dummy = 0;
     block_scan2(s_a, s_b, inc, dummy);
-    if (bt < p.BT) p.bt_chunk0[bt] = s_carry_a + inc - nch;
+    if (bt < p.BT) {
+      my_chunk0 = s_carry_a + inc - nch;
+      p.bt_chunk0[bt] = my_chunk0;
+    }
     __syncthreads();
     if (tid == kPlanThreads - 1) s_carry_a += inc;
     __syncthreads();
@@ -106,9 +112,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p) {
     const int bt = base + tid;
     int nseg = 0, nslot = 0, x = 0, e = 0;
     if (bt < p.BT) {
-      const int len = p.bt_len[bt];
+      const bool one_pass = p.BT <= kPlanThreads;
+      const int len = one_pass ? my_len : p.bt_len[bt];
       const int nch = (len + kChunk - 1) / kChunk;
-      x = p.bt_chunk0[bt];
+      x = one_pass ? my_chunk0 : p.bt_chunk0[bt];
       e = x + nch;
       if (nch > 0) nseg = 1 + starts_below(e, R, C) - starts_below(x + 1, R, C);
       nslot = nseg >= 2 ? nseg : 0;

@@ -28,7 +28,7 @@ constexpr int kWRows = 128;        // weight rows per CTA = MMA M
 constexpr int kMaxTokTile = 128;   // tokens per CTA at most = MMA N (TMEM columns)
 constexpr uint32_t kProjTmemCols = 128;
 constexpr int kSlab = 64;          // bf16 elements per 128-byte swizzled row
-constexpr int kOutTokTile = 64;    // tokens per CTA of the output kernel at most
+constexpr int kOutTokTile = 128;   // tokens per CTA of the output kernel at most
 constexpr int kRopeVec = 8;        // 16-byte pieces of q_rope a thread has in flight
 constexpr int kOutItems = kOutTokTile * 16 / 256;  // 8-float groups per thread and chunk
 
@@ -400,9 +400,9 @@ output_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const OutputArgs a) {
   if (warp == 1) tmem_free_cols(tmem);
 }
 
-// Tokens per CTA: enough token tiles that the grid covers the 148 SMs about twice, each a
-// multiple of 16 (the MMA's N step) and at most max_tile (128, the TMEM accumulator's columns,
-// for the query; 64 for the output, whose threads hold a chunk of the latent in registers).
+// Tokens per CTA of the absorbed query: enough token tiles that the grid covers the 148 SMs
+// about twice, each a multiple of 16 (the MMA's N step) and at most max_tile (the TMEM
+// accumulator's 128 columns).
 int token_tile(int n, int ctas_per_tile, int max_tile) {
   const int want = (2 * 148 + ctas_per_tile - 1) / ctas_per_tile;
   int tiles = (n + max_tile - 1) / max_tile;
@@ -458,7 +458,12 @@ cudaError_t launch_output_tc(const mla_config& c, const float* lat, const void* 
                              int n, uint32_t* err, cudaStream_t st) {
   const int H = c.num_heads, dv = c.head_dim_v, r = c.kv_rank;
   const int mts = (dv + kWRows - 1) / kWRows;
-  const int tile = token_tile(n, mts * H, kOutTokTile);
+  // every MMA instruction costs about the same whatever its N, and a CTA issues 2 r/16 of them
+  // (hi and lo terms), so the tokens are split over CTAs only as far as needed to keep each
+  // CTA's N at 128 or less
+  // (up to 64 tokens, two CTAs per head fill the SMs better than one)
+  const int tiles = n <= 64 ? (n + 31) / 32 : (n + kOutTokTile - 1) / kOutTokTile;
+  const int tile = std::min(kOutTokTile, round_up((n + tiles - 1) / tiles, 16));
   if (((uintptr_t)lat & 15) != 0) return cudaErrorInvalidValue;
   CUtensorMap tw;
   if (!make_bf16_map(&tw, w_uv, (uint64_t)r, (uint64_t)H * dv, (uint64_t)r * 2, kWRows))
