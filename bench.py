@@ -63,11 +63,12 @@ def aggregate_rate(units_per_rank_step: float, world: int, steps: int, elapsed_m
     return units_per_rank_step * world * steps / (elapsed_ms * 1e-3)
 
 
-# DRAM bytes (read + write) of one attention launch on the bench workload, from the ncu capture
-# summarised in profiles/step_kernels_dsv2.md, keyed by a hash of the kernel's sources: when the
-# kernel changes, the figure no longer applies and the bench reports null until it is re-measured.
+# DRAM bytes (read + write) of one attention launch on the bench workload, from an ncu capture
+# of that kernel source (profiles/attend_tc_dsv2.md), keyed by a hash of the kernel's sources:
+# when the kernel changes, the figure no longer applies and the bench reports null until it is
+# re-measured.
 ATTEND_SOURCES = ("decode_tc.cu", "tc_ptx.cuh", "tma_map.h", "common.cuh")
-ATTEND_TRAFFIC = {"79c3f674a9d716f4": 736_002_304 + 19_480_320}
+ATTEND_TRAFFIC = {"afc9c2737a02e388": 740_644_352 + 21_206_016}
 
 
 def attend_source_hash() -> str:

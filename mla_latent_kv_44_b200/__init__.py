@@ -14,6 +14,9 @@ import os
 from dataclasses import dataclass
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so")
+# The same library built with a test define that leaves out one K-slab load of the attention
+# kernel's first work range (tests of the bounded-wait path load it instead of LIB_PATH).
+TEST_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla_testhook.so")
 
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA, MLA_ERR_WORKSPACE = range(5)
 STATIC_WORKSPACE_BYTES = 40 << 20

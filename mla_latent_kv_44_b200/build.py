@@ -5,7 +5,9 @@
 Each csrc/*.cu compiles to an object under _build/ (recompiled when it or a header is newer),
 then the objects link into mla_latent_kv_44_b200/libmla.so with the CUDA runtime linked
 statically, so the library loads on a machine without a GPU (calls then fail with
-MLA_ERR_CUDA) and needs nothing at run time but the NVIDIA driver.
+MLA_ERR_CUDA) and needs nothing at run time but the NVIDIA driver. A second library,
+libmla_testhook.so, differs only in a test define of the attention kernel (one K-slab load of
+the first work range is left out); only the tests load it.
 """
 from __future__ import annotations
 
@@ -23,6 +25,11 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmla.so")
+# Test build: the same library with one K-slab load of the first work range left out
+# (MLA_TEST_DROP_ARRIVE), so that the tests can watch a bounded wait run out.
+TEST_LIB = os.path.join(PKG, "libmla_testhook.so")
+TEST_DEFINE = "-DMLA_TEST_DROP_ARRIVE"
+TEST_SOURCES = ("decode_tc.cu",)
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -37,7 +44,8 @@ def nvcc() -> str:
 
 
 def _headers():
-    return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
+    return (glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) +
+            glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def _stale(target: str, deps) -> bool:
@@ -54,6 +62,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     headers = _headers()
     jobs = []
     objs = []
+    test_objs = []
     for src in sources:
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
         objs.append(obj)
@@ -62,6 +71,13 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
             if ptxas_info:
                 cmd.insert(1, "-Xptxas=-v")
             jobs.append(cmd)
+        if os.path.basename(src) in TEST_SOURCES:
+            tobj = os.path.join(BUILD, os.path.basename(src) + ".testhook.o")
+            test_objs.append(tobj)
+            if force or _stale(tobj, [src] + headers):
+                jobs.append([cc, *ARCH, *FLAGS, TEST_DEFINE, "-c", src, "-o", tobj])
+        else:
+            test_objs.append(obj)
 
     def run(cmd):
         if verbose:
@@ -78,13 +94,14 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
                 failed.append(cmd[-3])
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(failed))
-    if force or jobs or _stale(LIB, objs):
-        cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs]
-        if verbose:
-            print(" ".join(cmd), flush=True)
-        p = subprocess.run(cmd, capture_output=True, text=True)
-        if p.returncode != 0:
-            raise RuntimeError("link failed:\n" + p.stdout + p.stderr)
+    for lib, parts in ((LIB, objs), (TEST_LIB, test_objs)):
+        if force or jobs or _stale(lib, parts):
+            cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-o", lib, *parts]
+            if verbose:
+                print(" ".join(cmd), flush=True)
+            p = subprocess.run(cmd, capture_output=True, text=True)
+            if p.returncode != 0:
+                raise RuntimeError("link failed:\n" + p.stdout + p.stderr)
     return LIB
 
 
