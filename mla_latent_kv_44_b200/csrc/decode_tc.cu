@@ -524,6 +524,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
     }
   } else if (warp == 0) {
     // ---------------------------------------------------------------- value: TMA producer
+    // This is the second and last read of these lines: evict them first, so that L2 keeps
+    // the score CTA's fresh loads, the partial outputs and the projection weights instead.
+    const uint64_t pol_drop = l2_evict_first();
     int vt = 0;
     bool ok = true;
     while (ok && walk.next(tl)) {
@@ -539,8 +542,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
           if (lane == 0) {
             mbar_expect_tx(bar(kVFull + vs), kVStageBytes);
             for (int i = 0; i < 4; ++i)
-              tma_load(s_base + kV_V + vs * kVStageBytes + i * kSlabBytes, &tm_kv,
-                       bar(kVFull + vs), 256 * dh + 64 * i, blk * kRows);
+              tma_load_hint(s_base + kV_V + vs * kVStageBytes + i * kSlabBytes, &tm_kv,
+                            bar(kVFull + vs), 256 * dh + 64 * i, blk * kRows, pol_drop);
           }
           __syncwarp();
         }
@@ -658,6 +661,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
         // O / l leaves through shared memory: each warp stages its 32 rows x 32 columns as a
         // 128-byte-swizzled 4 KB box and one lane stores the box with TMA, so the global
         // writes are whole lines rather than 16-byte pieces 2 KB apart.
+        // kept in L2: the combine (partials) and the output projection (O) read them next,
+        // after the rest of the cache has streamed through
+        const uint64_t keep = l2_evict_last();
         const CUtensorMap* map = tl.slot < 0 ? &tm_out : &tm_part;
         const int row0 = (tl.slot < 0 ? tl.bt : tl.slot) * kH + quad * 32;
         const uint32_t box = s_base + kV_Out + (uint32_t)quad * kOutBoxBytes;
@@ -681,7 +687,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
                          : "memory");
           fence_proxy_async();
           __syncwarp();
-          if (lane == 0) tma_store(map, box, 32 * ch, row0);
+          if (lane == 0) tma_store_hint(map, box, 32 * ch, row0, keep);
         }
         if (lane == 0) bulk_wait_read<0>();  // the box is free for the next segment
         __syncwarp();

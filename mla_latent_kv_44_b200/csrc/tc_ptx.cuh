@@ -71,6 +71,35 @@ __device__ __forceinline__ void tma_store(const CUtensorMap* map, uint32_t src, 
       "cp.async.bulk.commit_group;" ::"l"(map), "r"(src), "r"(x), "r"(y)
       : "memory");
 }
+// tma_store with an L2 cache policy (createpolicy) for the written lines
+__device__ __forceinline__ void tma_store_hint(const CUtensorMap* map, uint32_t src, int x, int y,
+                                               uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;\n\t"
+      "cp.async.bulk.commit_group;" ::"l"(map), "r"(src), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+// L2 policy that lets lines go before others (fraction 1.0)
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// tma_load with an L2 cache policy for the lines read
+__device__ __forceinline__ void tma_load_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                              int x, int y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y),
+      "l"(policy)
+      : "memory");
+}
+// L2 policy that keeps lines ahead of streaming data (fraction 1.0)
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
 // wait until at most N of this thread's bulk groups still read shared memory
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() {
