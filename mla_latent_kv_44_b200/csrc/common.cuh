@@ -33,7 +33,8 @@ struct WorkspaceLayout {
   size_t header;       // int32[64]: [0] segment count, [1] ranges used, [2] total chunks
   size_t range_begin;  // int32[kRanges + 1]: first segment of each range
   size_t segments;     // Segment[kRanges + BT]
-  size_t bt_first;     // int32[BT]: first segment of each row group
+  size_t bt_slot0;     // int32[BT]: first partial slot of a split row group (its slots are
+                       // consecutive), -1 for a row group in one segment
   size_t bt_nseg;      // int32[BT]: number of segments of each row group (0: invalid length)
   size_t bt_len;       // int32[BT]: rows attended by each row group
   size_t bt_chunk0;    // int32[BT]: exclusive prefix of chunk counts
@@ -51,7 +52,7 @@ inline WorkspaceLayout workspace_layout(int H, int r, int bt_count) {
   L.header = take(64 * sizeof(int32_t));
   L.range_begin = take((kRanges + 1) * sizeof(int32_t));
   L.segments = take(size_t(kRanges + bt_count) * sizeof(Segment));
-  L.bt_first = take(size_t(bt_count) * sizeof(int32_t));
+  L.bt_slot0 = take(size_t(bt_count) * sizeof(int32_t));
   L.bt_nseg = take(size_t(bt_count) * sizeof(int32_t));
   L.bt_len = take(size_t(bt_count) * sizeof(int32_t));
   L.bt_chunk0 = take(size_t(bt_count) * sizeof(int32_t));
@@ -74,7 +75,7 @@ struct DecodeParams {
   int32_t* header;
   int32_t* range_begin;
   Segment* segments;
-  int32_t* bt_first;
+  int32_t* bt_slot0;
   int32_t* bt_nseg;
   int32_t* bt_len;
   int32_t* bt_chunk0;

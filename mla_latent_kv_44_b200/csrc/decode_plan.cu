@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p) {
     if (bt < p.BT) {
       const int first = s_carry_a + inc_seg - nseg;
       const int slot0 = s_carry_b + inc_slot - nslot;
-      p.bt_first[bt] = first;
+      p.bt_slot0[bt] = nseg >= 2 ? slot0 : -1;
       p.bt_nseg[bt] = nseg;
       // cut points of this row group: x, the range starts strictly inside (x, e), e
       int q = starts_below(x + 1, R, C);  // first range starting after x
@@ -171,22 +171,19 @@ cudaError_t launch_plan(const DecodeParams& p, cudaStream_t st) {
 constexpr int kCombineHeads = 4;
 
 __global__ void __launch_bounds__(kCombineHeads * 32) combine_kernel(DecodeParams p) {
-  __shared__ int s_slot[kRanges];
   __shared__ float s_w[kCombineHeads][kRanges];
   const int bt = blockIdx.x;
   wait_prior_grid();
   const int nseg = p.bt_nseg[bt];
+  const int slot0 = p.bt_slot0[bt];  // a split row group's slots are slot0 .. slot0 + nseg - 1
   if (nseg == 1) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y * kCombineHeads + warp;
-  const int first = p.bt_first[bt];
-  for (int k = threadIdx.x; k < nseg; k += blockDim.x) s_slot[k] = p.segments[first + k].slot;
-  __syncthreads();
   if (h >= p.H) return;
   float4* dst = (float4*)(p.out + ((size_t)bt * p.H + h) * p.r);
   const int r4 = p.r / 4;
   float mx = -INFINITY;
-  for (int k = lane; k < nseg; k += 32) mx = fmaxf(mx, p.part_lse[(size_t)s_slot[k] * p.H + h]);
+  for (int k = lane; k < nseg; k += 32) mx = fmaxf(mx, p.part_lse[(size_t)(slot0 + k) * p.H + h]);
   mx = warp_max(mx);
   if (nseg == 0 || mx == -INFINITY) {  // no rows (bad length, or every block rejected)
     for (int d = lane; d < r4; d += 32) dst[d] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -194,11 +191,11 @@ __global__ void __launch_bounds__(kCombineHeads * 32) combine_kernel(DecodeParam
     return;
   }
   float z = 0.f;
-  for (int k = lane; k < nseg; k += 32) z += expf(p.part_lse[(size_t)s_slot[k] * p.H + h] - mx);
+  for (int k = lane; k < nseg; k += 32) z += expf(p.part_lse[(size_t)(slot0 + k) * p.H + h] - mx);
   z = warp_sum(z);
   const float L = mx + logf(z);
   for (int k = lane; k < nseg; k += 32)
-    s_w[warp][k] = expf(p.part_lse[(size_t)s_slot[k] * p.H + h] - L);
+    s_w[warp][k] = expf(p.part_lse[(size_t)(slot0 + k) * p.H + h] - L);
   __syncwarp();
   // a lane holds up to four float4 of the row at once (r = 512 in one pass), so every partial's
   // loads for the whole row are in flight together
@@ -209,7 +206,7 @@ __global__ void __launch_bounds__(kCombineHeads * 32) combine_kernel(DecodeParam
 #pragma unroll 2
     for (int k = 0; k < nseg; ++k) {
       const float w = s_w[warp][k];
-      const float4* src = (const float4*)(p.part_o + ((size_t)s_slot[k] * p.H + h) * p.r);
+      const float4* src = (const float4*)(p.part_o + ((size_t)(slot0 + k) * p.H + h) * p.r);
       float4 v[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u)

@@ -667,14 +667,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
         const CUtensorMap* map = tl.slot < 0 ? &tm_out : &tm_part;
         const int row0 = (tl.slot < 0 ? tl.bt : tl.slot) * kH + quad * 32;
         const uint32_t box = s_base + kV_Out + (uint32_t)quad * kOutBoxBytes;
+        // the next chunk's TMEM load is in flight while this chunk is staged and stored
+        uint32_t o[32], nx[32];
+        tmem_ld32(tq, o);
 #pragma unroll 1
         for (int ch = 0; ch < 16; ++ch) {
+          if (ch + 1 < 16) tmem_ld32_async(tq + 32 * (ch + 1), nx);
           if (ch >= 1) {  // the previous chunk's store is done reading the box
             if (lane == 0) bulk_wait_read<0>();
             __syncwarp();
           }
-          uint32_t o[32];
-          tmem_ld32(tq + 32 * ch, o);
           const uint32_t row = box + (uint32_t)lane * 128;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
@@ -688,6 +690,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
           fence_proxy_async();
           __syncwarp();
           if (lane == 0) tma_store_hint(map, box, 32 * ch, row0, keep);
+          if (ch + 1 < 16) {
+            tmem_wait_ld(nx);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = nx[i];
+          }
         }
         if (lane == 0) bulk_wait_read<0>();  // the box is free for the next segment
         __syncwarp();

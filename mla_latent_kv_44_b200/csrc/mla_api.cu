@@ -132,7 +132,7 @@ mla_status mla_decode_stages(const mla_config* cfg, int32_t stages, const void* 
   p.header = reinterpret_cast<int32_t*>(ws + L.header);
   p.range_begin = reinterpret_cast<int32_t*>(ws + L.range_begin);
   p.segments = reinterpret_cast<Segment*>(ws + L.segments);
-  p.bt_first = reinterpret_cast<int32_t*>(ws + L.bt_first);
+  p.bt_slot0 = reinterpret_cast<int32_t*>(ws + L.bt_slot0);
   p.bt_nseg = reinterpret_cast<int32_t*>(ws + L.bt_nseg);
   p.bt_len = reinterpret_cast<int32_t*>(ws + L.bt_len);
   p.bt_chunk0 = reinterpret_cast<int32_t*>(ws + L.bt_chunk0);
