@@ -28,6 +28,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MLA absorbed decode: cache TB/s (frac of HBM/MMA roofline), tokens/s, B=64 S=8k"
 REF_BUDGET_S = 150.0  # whole --impl reference run
+DATASHEET_HBM_GBS = 8000.0
+DATASHEET_BF16_TFLOPS = 2250.0
 
 
 def parse():
@@ -492,7 +494,24 @@ def run_ours(args, w):
                  "avg_launch_us": attend_ms * 1e3, "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"
                  if peak_src == "measured" else "fallback",
                  "tensor_view": {"achieved_tflops": tflops, "peak": tc_burst,
-                                 "frac": tflops / tc_burst}})
+                                 "frac": tflops / tc_burst},
+                 # the same achieved rates against the datasheet figures (about 8 TB/s HBM3e,
+                 # 2.25 PFLOP/s dense bf16), for context
+                 "frac_datasheet": {"hbm": gbs / DATASHEET_HBM_GBS,
+                                    "tensor": tflops / DATASHEET_BF16_TFLOPS}})
+    # per-stage rates of the projections and the append (algorithmic bytes and FLOPs over the
+    # per-kernel times of the breakdown run)
+    N, H = tokens_per_step, w.num_heads
+    stage_work = {
+        "absorb": (H * w.head_dim * w.kv_rank * 2 + N * H * (w.head_dim + w.rope_dim) * 2 +
+                   N * H * w.row_width * 2, 2 * N * H * w.head_dim * w.kv_rank),
+        "append": (N * (w.row_width * 2 + w.kv_rank * 4) + N * w.row_width * 2, 0),
+        "output": (H * w.head_dim_v * w.kv_rank * 2 + N * H * w.kv_rank * 4 +
+                   N * H * w.head_dim_v * 2, 2 * N * H * w.head_dim_v * w.kv_rank),
+    }
+    stages_rate = {k: {"GB/s": b / (stage_ms[k] * 1e-3) / 1e9,
+                       "GFLOP/s": f / (stage_ms[k] * 1e-3) / 1e9}
+                   for k, (b, f) in stage_work.items()}
     ms_per_step = elapsed_ms / args.steps
     value = aggregate_rate(tokens_per_step, world, args.steps, elapsed_ms)
     e2e_value = aggregate_rate(tokens_per_step, world, e2e_steps, e2e_ms)
@@ -512,6 +531,7 @@ def run_ours(args, w):
         "stages_us": {k: v * 1e3 for k, v in stage_ms.items()},
         "stages_note": ("per-kernel times from a separate run with an event after every kernel; "
                         "the timed steps chain the kernels with programmatic dependent launch"),
+        "stages_rate": stages_rate,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": 6 * args.steps,
