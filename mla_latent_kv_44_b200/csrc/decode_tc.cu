@@ -49,6 +49,8 @@ constexpr unsigned long long kTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int kKStages = 4;
 constexpr int kKStageBytes = kTileBlocks * kSlabBytes;        // 32 KB
 constexpr int kQRopeBytes = kH * 64 * 2;                      // 16 KB
+constexpr int kQBoxBytes = kH * 64 * 2;                       // 128 heads x 64 dims
+constexpr int kQStages = kR / 128;                            // ring uses for Q's latent part
 constexpr int kPBlockBytes = kH * kRows * 2;                  // 128 x 64 bf16: 16 KB
 constexpr int kHdrBytes = 2 * kH * 4;                         // alpha[128], l[128]
 constexpr int kS_K = 0;
@@ -75,7 +77,7 @@ enum Bar {
   // score CTA
   kKFull = 0,
   kKEmpty = kKFull + kKStages,
-  kQFull = kKEmpty + kKStages,  // Q of the segment in place (TMA RoPE part + 4 softmax warps)
+  kQFull = kKEmpty + kKStages,  // RoPE part of the segment's Q in shared memory
   kQEmpty,                      // last S product of the segment done with Q
   kSFull,                       // S complete
   kSFree,                       // softmax done reading S
@@ -107,8 +109,9 @@ struct Ctl {
   volatile int* abort;
 };
 
-// Warp-collective bounded wait; the result is the same in all 32 lanes.
-__device__ __noinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Ctl& c) {
+// Warp-collective bounded wait; the result is the same in all 32 lanes. The first poll is
+// inlined: with a call at every wait the kernel ran about 10% slower.
+__device__ __noinline__ bool warp_wait_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
   uint64_t t0 = 0;
   for (int it = 0;; ++it) {
     const bool done = mbar_try(bar, parity);
@@ -124,6 +127,10 @@ __device__ __noinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Ctl&
       return false;
     }
   }
+}
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Ctl& c) {
+  if (__all_sync(0xffffffffu, mbar_try(bar, parity))) return true;
+  return warp_wait_slow(bar, parity, c);
 }
 
 // Barrier of a group of warps on an mbarrier that counts one arrival per warp: the k-th use
@@ -217,7 +224,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
         mbar_init(bar(kKFull + i), 1);
         mbar_init(bar(kKEmpty + i), 1);
       }
-      mbar_init(bar(kQFull), 9);
+      mbar_init(bar(kQFull), 1);
       mbar_init(bar(kQEmpty), 1);
       mbar_init(bar(kSFull), 1);
       mbar_init(bar(kSFree), 8);
@@ -276,7 +283,27 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
     int kt = 0, seg_i = 0;
     bool ok = true;
     while (ok && walk.next(tl)) {
-      if (tl.first) {  // RoPE part of Q for this segment, once the previous segment's S is done
+      if (tl.first) {
+        // Q's latent part passes through the K ring (two 64-dim boxes of 128 heads per stage);
+        // the MMA warp copies it into TMEM. The ring keeps streaming: these loads only wait
+        // for stages that the previous segment's last products have released.
+        for (int qs = 0; qs < kQStages && ok; ++qs, ++kt) {
+          const int stage = kt % kKStages;
+          if (kt >= kKStages &&
+              !warp_wait(bar(kKEmpty + stage), ((kt / kKStages) - 1) & 1, ctl)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            mbar_expect_tx(bar(kKFull + stage), kKStageBytes);
+            for (int b = 0; b < 2; ++b)
+              tma_load(s_base + kS_K + stage * kKStageBytes + b * kQBoxBytes, &tm_q,
+                       bar(kKFull + stage), 64 * (2 * qs + b), tl.bt * kH);
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        // RoPE part of Q into its own buffer, once the previous segment's S is done with it
         if (seg_i > 0 && !warp_wait(bar(kQEmpty), (seg_i - 1) & 1, ctl)) break;
         if (lane == 0) {
           mbar_expect_tx(bar(kQFull), kQRopeBytes);
@@ -317,12 +344,38 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
     bool ok = true;
     while (ok && walk.next(tl)) {
       if (tl.first) {
-        ok = warp_wait(bar(kQFull), seg_i & 1, ctl);
+        // the previous segment's S products have finished reading Q from TMEM
+        if (seg_i > 0) ok = warp_wait(bar(kQEmpty), (seg_i - 1) & 1, ctl);
+        // Q's latent part, staged by TMA in the K ring, into TMEM columns 256..511 (head h
+        // in lane h, dims 2c and 2c + 1 in column 256 + c): 16 dims per copy, from the same
+        // K-major 128-byte-swizzled layout an MMA operand descriptor reads. Copies and the
+        // MMAs after them are issued by this thread and execute in order.
+        for (int qs = 0; qs < kQStages && ok; ++qs, ++kt) {
+          const int stage = kt % kKStages;
+          if (!warp_wait(bar(kKFull + stage), (kt / kKStages) & 1, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_after();
+          if (lane == 0) {
+            const uint32_t sb = s_base + kS_K + stage * kKStageBytes;
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                tmem_cp128x256b(tmem + 256 + 32 * (2 * qs + b) + 8 * i,
+                                sdesc(sb + b * kQBoxBytes + 32 * i, 16, 1024, 2));
+            tc_commit(bar(kKEmpty + stage));
+          }
+          __syncwarp();
+        }
+        if (ok) ok = warp_wait(bar(kQFull), seg_i & 1, ctl);
         ++seg_i;
       }
       if (ok && t > 0) ok = warp_wait(bar(kSFree), (t - 1) & 1, ctl);
       if (!ok) break;
       const uint32_t id = idesc(128, kRows * tl.nb, 0);
+#pragma unroll
       for (int k = 0; k < 9; ++k, ++kt) {
         const int stage = kt % kKStages;
         if (!warp_wait(bar(kKFull + stage), (kt / kKStages) & 1, ctl)) {
@@ -363,50 +416,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
     const int h = quad * 32 + lane;
     const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
     const float c2 = p.scale * 1.4426950408889634f;  // scores in log2 units
-    const __nv_bfloat16* Q = (const __nv_bfloat16*)p.q;
     const uint32_t stage_p = s_base + kS_Stage;
     const uint32_t hdr = s_base + kS_Hdr;
     float* red = (float*)(smem + kS_Red);  // [0..255]: max of half 0 / 1; [256..511]: sums
 
-    auto load_qckv = [&](int bt) {  // this warp's half of Q's latent part into TMEM
-      const uint4* src = (const uint4*)(Q + ((size_t)bt * kH + h) * kD);
-#pragma unroll 1
-      for (int ch = 4 * half; ch < 4 * half + 4; ch += 2) {  // 512 bytes of the row in flight
-        uint4 x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = src[8 * ch + i];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t w[32];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            w[4 * i] = x[8 * c + i].x; w[4 * i + 1] = x[8 * c + i].y;
-            w[4 * i + 2] = x[8 * c + i].z; w[4 * i + 3] = x[8 * c + i].w;
-          }
-          tmem_st32(tq + 256 + 32 * (ch + c), w);
-        }
-      }
-      tmem_wait_st();
-      tc_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kQFull));
-    };
-
     int t = 0;
     float m_ref = 0.f, l = 0.f;
-    bool ok = true, q_loaded = false;
+    bool ok = true;
     while (ok && walk.next(tl)) {
-      if (!q_loaded) {
-        load_qckv(tl.bt);
-        q_loaded = true;
-      }
       if (!warp_wait(bar(kSFull), t & 1, ctl)) break;
       tc_after();
-      if (tl.last) {  // the segment's last S product is done: bring in the next query
-        TileWalk look = walk;
-        Tile nx;
-        if (look.next(nx)) load_qckv(nx.bt);
-      }
       uint32_t v[128];
       tmem_ld128(tq + 128 * half, v);
       tc_before();

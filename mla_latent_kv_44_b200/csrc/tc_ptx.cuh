@@ -256,6 +256,13 @@ __device__ __forceinline__ void mma_ss(uint32_t d, uint64_t adesc, uint64_t bdes
       "l"(bdesc), "r"(id), "r"(acc)
       : "memory");
 }
+// TMEM[lanes 0..127, 8 columns from taddr] = the 128 x 32-byte matrix the descriptor names
+// (asynchronous like an MMA: ordered before later MMAs of the issuing thread, tracked by
+// tc_commit)
+__device__ __forceinline__ void tmem_cp128x256b(uint32_t taddr, uint64_t sdesc_src) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc_src)
+               : "memory");
+}
 // shared::cta -> peer shared::cluster bulk copy, completing bytes on the peer's mbarrier
 __device__ __forceinline__ void bulk_to_peer(uint32_t dst, uint32_t src, uint32_t bytes,
                                              uint32_t peer_bar) {
