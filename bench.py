@@ -70,7 +70,7 @@ def aggregate_rate(units_per_rank_step: float, world: int, steps: int, elapsed_m
 # when the kernel changes, the figure no longer applies and the bench reports null until it is
 # re-measured.
 ATTEND_SOURCES = ("decode_tc.cu", "tc_ptx.cuh", "tma_map.h", "common.cuh")
-ATTEND_TRAFFIC = {"650ea39a8618bb01": 646_682_112 + 8_925_184}
+ATTEND_TRAFFIC = {"6adc85654eda141d": 646_193_152 + 8_178_176}
 
 
 def attend_source_hash() -> str:
