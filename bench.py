@@ -66,20 +66,25 @@ def aggregate_rate(units_per_rank_step: float, world: int, steps: int, elapsed_m
 
 
 # DRAM bytes (read + write) of one attention launch on the bench workload, from an ncu capture
-# of that kernel source (profiles/attend_tc_dsv2.md), keyed by a hash of the kernel's sources:
+# of that kernel source (profiles/attend_tc_dsv2.md), keyed by a hash of the kernel's code:
 # when the kernel changes, the figure no longer applies and the bench reports null until it is
 # re-measured.
 ATTEND_SOURCES = ("decode_tc.cu", "tc_ptx.cuh", "tma_map.h", "common.cuh")
-ATTEND_TRAFFIC = {"6adc85654eda141d": 646_193_152 + 8_178_176}
+ATTEND_TRAFFIC = {"483f7328a205a490": 646_193_152 + 8_178_176}
 
 
 def attend_source_hash() -> str:
+    """Hash of the attention kernel's code: comments and whitespace do not count."""
     import hashlib
+    import re
 
     h = hashlib.sha256()
     for f in ATTEND_SOURCES:
-        with open(os.path.join(ROOT, "mla_latent_kv_44_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "mla_latent_kv_44_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -14,7 +14,9 @@
 // the two CTAs of a cluster take different roles for each work range:
 //   * the score CTA keeps the latent part of Q in TMEM (256 columns, A operand) and its RoPE
 //     part in shared memory, streams the cache rows' 64-dim slabs by TMA and accumulates S in
-//     the other 256 TMEM columns. Eight softmax warps copy S into registers (128 values per
+//     the other 256 TMEM columns. At each segment start Q's latent part comes through the same
+//     TMA ring as the cache slabs and the MMA warp copies it into TMEM (tcgen05.cp), so a
+//     switch to the next sequence costs the score CTA about one ring refill. Eight softmax warps copy S into registers (128 values per
 //     thread) and release it at once, so the next tile's S = Q . K^T runs on the tensor core
 //     while this tile's online softmax runs (exp2 units, O rescaled lazily only when the
 //     running max grows by more than 2^8). P (bf16) and the per-row rescale factors and sums
