@@ -304,6 +304,47 @@ def run_reference(args, w):
 # ---------------------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------------------
+def attention_roofline(w, rows, attend_ms: float, peaks, traffic):
+    """Roofline object of the attention kernel for one launch over ``rows`` cached rows.
+
+    Algorithmic work per attended row and query token, all heads: the 576-value row read once
+    (1152 B in bf16) and 2 * H * (576 + 512) FLOP. ``peaks`` is load_peaks()'s tuple; ``traffic``
+    the captured DRAM bytes of this kernel source or None. Returns (roofline dict, algorithmic
+    bytes, achieved GB/s, achieved TFLOP/s).
+    """
+    T = w.new_tokens
+    attended = int(sum(int(n) - T + 1 + t_ for n in rows for t_ in range(T)))
+    row_bytes = w.row_width * 2
+    flops_row = w.num_heads * 2 * (w.row_width + w.kv_rank)
+    attend_bytes = attended * row_bytes
+    attend_flops = attended * flops_row
+    hbm, tc_burst, _tc_sust, peak_src = peaks
+    attend_s = attend_ms * 1e-3
+    gbs = attend_bytes / attend_s / 1e9
+    tflops = attend_flops / attend_s / 1e12
+    bound = "hbm" if attend_bytes / (hbm * 1e9) >= attend_flops / (tc_burst * 1e12) else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}
+    else:
+        roof = {"bound": "tensor", "achieved": tflops, "peak": tc_burst, "unit": "TFLOP/s",
+                "frac": tflops / tc_burst}
+    roof.update({"traffic": traffic, "kernel": "mla attention (split-KV main)",
+                 "traffic_note": ("DRAM read+write bytes per launch from one ncu capture of this "
+                                  "kernel source (cold L2); algorithmic bytes are %d" % attend_bytes)
+                 if traffic else "no ncu capture of this kernel source",
+                 "algorithmic_bytes_per_launch": attend_bytes,
+                 "algorithmic_flops_per_launch": attend_flops,
+                 "avg_launch_us": attend_ms * 1e3, "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"
+                 if peak_src == "measured" else "fallback",
+                 "tensor_view": {"achieved_tflops": tflops, "peak": tc_burst,
+                                 "frac": tflops / tc_burst},
+                 # the same achieved rates against the datasheet figures (about 8 TB/s HBM3e,
+                 # 2.25 PFLOP/s dense bf16), for context
+                 "frac_datasheet": {"hbm": gbs / DATASHEET_HBM_GBS,
+                                    "tensor": tflops / DATASHEET_BF16_TFLOPS}})
+    return roof, attend_bytes, gbs, tflops
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -474,36 +515,8 @@ def run_ours(args, w):
     import mla_inputs as mi
 
     rows = mi.total_rows(w, 0)
-    attended = int(sum(int(n) - T + 1 + t_ for n in rows for t_ in range(T)))
-    row_bytes = w.row_width * 2
-    flops_row = w.num_heads * 2 * (w.row_width + w.kv_rank)
-    attend_bytes = attended * row_bytes
-    attend_flops = attended * flops_row
-    hbm, tc_burst, tc_sust, peak_src = load_peaks()
-    attend_s = attend_ms * 1e-3
-    gbs = attend_bytes / attend_s / 1e9
-    tflops = attend_flops / attend_s / 1e12
-    bound = "hbm" if attend_bytes / (hbm * 1e9) >= attend_flops / (tc_burst * 1e12) else "tensor"
-    if bound == "hbm":
-        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}
-    else:
-        roof = {"bound": "tensor", "achieved": tflops, "peak": tc_burst, "unit": "TFLOP/s",
-                "frac": tflops / tc_burst}
-    traffic = ATTEND_TRAFFIC.get(attend_source_hash())
-    roof.update({"traffic": traffic, "kernel": "mla attention (split-KV main)",
-                 "traffic_note": ("DRAM read+write bytes per launch from one ncu capture of this "
-                                  "kernel source (cold L2); algorithmic bytes are %d" % attend_bytes)
-                 if traffic else "no ncu capture of this kernel source",
-                 "algorithmic_bytes_per_launch": attend_bytes,
-                 "algorithmic_flops_per_launch": attend_flops,
-                 "avg_launch_us": attend_ms * 1e3, "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"
-                 if peak_src == "measured" else "fallback",
-                 "tensor_view": {"achieved_tflops": tflops, "peak": tc_burst,
-                                 "frac": tflops / tc_burst},
-                 # the same achieved rates against the datasheet figures (about 8 TB/s HBM3e,
-                 # 2.25 PFLOP/s dense bf16), for context
-                 "frac_datasheet": {"hbm": gbs / DATASHEET_HBM_GBS,
-                                    "tensor": tflops / DATASHEET_BF16_TFLOPS}})
+    roof, attend_bytes, gbs, tflops = attention_roofline(w, rows, attend_ms, load_peaks(),
+                                                         ATTEND_TRAFFIC.get(attend_source_hash()))
     # per-stage rates of the projections and the append (algorithmic bytes and FLOPs over the
     # per-kernel times of the breakdown run)
     N, H = tokens_per_step, w.num_heads

@@ -82,3 +82,43 @@ def test_clock_summary_falls_back_to_the_nearest_samples_for_a_short_region():
 def test_clock_summary_without_samples_reports_none():
     got = _sampler([]).summary(0.0, 1.0)
     assert got["sm_mhz"] is None and got["samples"] == 0
+
+
+def test_attention_roofline_counts_the_algorithmic_bytes_and_flops():
+    import mla_inputs as mi
+
+    w = mi.WORKLOADS["dsv2"]
+    rows = mi.total_rows(w, 0)
+    peaks = (6538.9, 1608.2, None, "measured")
+    roof, nbytes, gbs, tflops = bench.attention_roofline(w, rows, 0.2, peaks, None)
+    # 64 sequences of 8192 cached rows + the new one; 1152 B and 2*128*(576+512) FLOP per row
+    assert nbytes == 64 * 8193 * 1152 == roof["algorithmic_bytes_per_launch"]
+    assert roof["algorithmic_flops_per_launch"] == 64 * 8193 * 278_528
+    # at these peaks the byte time (92.4 us) exceeds the FLOP time (90.8 us): HBM-bound
+    assert roof["bound"] == "hbm" and roof["unit"] == "GB/s"
+    assert gbs == pytest.approx(nbytes / 0.2e-3 / 1e9)
+    assert roof["frac"] == pytest.approx(gbs / 6538.9)
+    assert roof["tensor_view"]["achieved_tflops"] == pytest.approx(tflops)
+    assert roof["traffic"] is None and roof["avg_launch_us"] == pytest.approx(200.0)
+
+
+def test_attention_roofline_counts_causal_rows_per_query_token():
+    import mla_inputs as mi
+
+    w = mi.WORKLOADS["mtp"]
+    rows = mi.total_rows(w, 0)
+    _, nbytes, _, _ = bench.attention_roofline(w, rows, 1.0, (6538.9, 1608.2, None, "x"), 1)
+    # 32 sequences of 16384 cached rows and 4 new tokens: token t sees 16384 + t + 1 rows
+    assert len(rows) == 32 and all(int(n) == 16384 + 4 for n in rows)
+    assert nbytes == 32 * (16385 + 16386 + 16387 + 16388) * 1152 == 2_416_287_744
+
+
+def test_attention_roofline_switches_to_tensor_when_bytes_are_cheap():
+    import mla_inputs as mi
+
+    w = mi.WORKLOADS["dsv2"]
+    roof, _, _, tflops = bench.attention_roofline(w, mi.total_rows(w, 0), 0.2,
+                                                  (20000.0, 1608.2, None, "measured"), 123)
+    assert roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
+    assert roof["frac"] == pytest.approx(tflops / 1608.2)
+    assert roof["traffic"] == 123
