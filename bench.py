@@ -66,7 +66,7 @@ def aggregate_rate(units_per_rank_step: float, world: int, steps: int, elapsed_m
 
 
 # DRAM bytes (read + write) of one attention launch on the bench workload, from an ncu capture
-# of that kernel source (profiles/attend_tc_dsv2.md), keyed by a hash of the kernel's code:
+# of that kernel source, keyed by a hash of the kernel's code:
 # when the kernel changes, the figure no longer applies and the bench reports null until it is
 # re-measured.
 ATTEND_SOURCES = ("decode_tc.cu", "tc_ptx.cuh", "tma_map.h", "common.cuh")

@@ -192,8 +192,8 @@ MLA_API mla_status mla_decode_static_workspace(const mla_config* cfg, const void
                                                uint32_t* dev_err, void* stream);
 
 /*
- * mla_output -- [B] Absorbing projections, [C] "rearrangement for calculating the final
- * output": o[n, h, :] = W_UV[h] out_latent[n, h, :] (fp32 accumulation).
+ * mla_output -- [B] Absorbing projections, [C] the output rearrangement figure (W_UV applied
+ * after the weighted sum): o[n, h, :] = W_UV[h] out_latent[n, h, :] (fp32 accumulation).
  * out_latent (n_tokens, H, r) float32; w_uv (H, d_v, r) dtype (the nn.Linear(r, H*d_v)
  * weight); o (n_tokens, H, d_v) dtype. W_O is not part of the library.
  * For bf16 the tensor-core kernel feeds out_latent to its bf16 MMA as two terms, hi = bf16(x)

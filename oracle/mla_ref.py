@@ -66,9 +66,9 @@ def rope_inv_freq(d_r: int, base: float) -> np.ndarray:
 def rope_rotate(x: np.ndarray, pos, base: float) -> np.ndarray:
     """Rotate adjacent pairs (x[2i], x[2i+1]) of the last axis by the angle pos * theta_i.
 
-    "Build a DeepSeek Model from Scratch" ch. 3, figures "The dimensions of a Query or Key
-    vector are paired up for rotation" and "Each pair of dimensions is treated as a 2D vector
-    and rotated by a position-dependent angle". ``pos`` broadcasts against x.shape[:-1].
+    "Build a DeepSeek Model from Scratch" ch. 3, the two RoPE figures (a query or key vector's
+    dimensions taken two at a time, each pair turned as a 2-D vector through an angle that
+    grows with the position). ``pos`` broadcasts against x.shape[:-1].
     """
     x = np.asarray(x)
     d_r = x.shape[-1]
@@ -207,13 +207,6 @@ def append_ref(pool: np.ndarray, ckv_raw, krope_raw, gamma, seq_idx, pos, table,
     return pl
 
 
-def gather_sequence(pool: np.ndarray, table_row: np.ndarray, length: int) -> np.ndarray:
-    """Rows 0..length-1 of one sequence, read back through its block table."""
-    bs = pool.shape[1]
-    pos = np.arange(length)
-    return pool[table_row[pos // bs], pos % bs]
-
-
 # --------------------------------------------------------------------------------------
 # Attention: naive form (the authority) and absorbed form
 # --------------------------------------------------------------------------------------
@@ -237,8 +230,9 @@ def naive_decode(c_kv: np.ndarray, k_rope: np.ndarray, q_nope: np.ndarray, q_rop
     v = W_UV(c_kv_full) reshaped per head, attn = softmax(q k^T * scale) with the causal
     mask for several query tokens, out = attn v. "Multi-head latent attention",
     ``_project_mla``: the key is [k_content || k_rope] with the RoPE key broadcast to every
-    head; the query is [q_nope || q_rope]. "Build a DeepSeek Model from Scratch" ch. 3:
-    "Decompressing the updated latent cache into the full Key and Value matrices".
+    head; the query is [q_nope || q_rope]. "Build a DeepSeek Model from Scratch" ch. 3, the
+    cache-update figure: the whole updated latent cache is expanded into full per-head keys
+    and values before the attention.
 
     c_kv (L, r) and k_rope (L, d_r) hold every row including the T new ones (already normed
     and rotated); q_nope (T, H, d_h), q_rope (T, H, d_r) rotated; w_uk (H, d_h, r) and
@@ -351,7 +345,8 @@ def output_ref(o_lat: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
     """o[n, h] = W_UV[h] o_lat[n, h]: the value up-projection applied after the weighted sum.
 
     "MLA from scratch in PyTorch", Absorbing projections; "Build a DeepSeek Model from
-    Scratch" ch. 3, "The mathematical rearrangement for calculating the final output in MLA".
+    Scratch" ch. 3, the figure on the output rearrangement (W_UV applied after the weighted
+    sum).
     o_lat (N, H, r), w_uv (H, d_v, r) -> (N, H, d_v).
     """
     return np.einsum("hij,nhj->nhi", np.asarray(w_uv, dtype=F64), np.asarray(o_lat, dtype=F64))

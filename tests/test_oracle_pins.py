@@ -64,9 +64,58 @@ def test_decode_work_per_row():
     # 576-wide bf16 row = 1152 B; 128 heads x 2 x (576 + 512) FLOPs.
     nbytes, flops = acc.absorbed_decode_work(1, 128, 512, 64)
     assert nbytes == 1152 and flops == 278528
-    # the naive form's up-projection dominates its FLOPs (what absorption removes)
-    naive = acc.naive_decode_flops(4096, 128, 128, 512)
-    assert naive == 2 * 2 * 4096 * 512 * 128 * 128 + 2 * 128 * 128 * 4096
+
+
+class _CountingFloat:
+    """A float that counts the multiplications and additions performed on it."""
+    mul = 0
+    add = 0
+
+    def __init__(self, v):
+        self.v = float(v)
+
+    def __mul__(self, o):
+        _CountingFloat.mul += 1
+        return _CountingFloat(self.v * (o.v if isinstance(o, _CountingFloat) else o))
+
+    def __add__(self, o):
+        _CountingFloat.add += 1
+        return _CountingFloat(self.v + (o.v if isinstance(o, _CountingFloat) else o))
+
+
+def test_naive_decode_flops_counts_the_contractions_of_the_expanded_form():
+    # "MLA from scratch in PyTorch", The up-projection cost at decode time: the expanded form
+    # rebuilds K and V from every cached latent, then scores the query against K. Count the
+    # multiply-adds a scalar-loop version of exactly those contractions executes at a tiny
+    # shape (one multiply and one add per term, 2 FLOPs per multiply-add, as the page counts),
+    # check that the loops compute the oracle's K, V and scores, and compare the count.
+    S, H, dh, r = 5, 3, 2, 4
+    g = np.random.default_rng([5, 1])
+    c = g.standard_normal((S, r))
+    wuk = g.standard_normal((H, dh, r))
+    wuv = g.standard_normal((H, dh, r))
+    q = g.standard_normal((H, dh))
+    C = _CountingFloat
+    C.mul = C.add = 0
+
+    def dot(a, b):
+        acc_ = C(0.0)
+        for x, y in zip(a, b):
+            acc_ = acc_ + C(x) * y
+        return acc_.v
+
+    K = np.array([[[dot(wuk[h, i], c[j]) for i in range(dh)] for j in range(S)] for h in range(H)])
+    V = np.array([[[dot(wuv[h, i], c[j]) for i in range(dh)] for j in range(S)] for h in range(H)])
+    s = np.array([[dot(q[h], K[h, j]) for j in range(S)] for h in range(H)])
+    assert C.mul == C.add
+    counted = 2 * C.mul
+    assert counted == acc.naive_decode_flops(S, H, dh, r)
+    # the loops are the expanded form's own contractions
+    np.testing.assert_allclose(K, np.einsum("hir,jr->hji", wuk, c), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(V, np.einsum("hir,jr->hji", wuv, c), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(s, np.einsum("hi,hji->hj", q, K), rtol=1e-12, atol=1e-12)
+    # and an asymmetric shape cannot pass with d_h and r exchanged in only one of the terms
+    assert acc.naive_decode_flops(S, H, dh, r) != 4 * S * r * H * dh + 2 * H * r * S
 
 
 # ----------------------------------------------------------------------------------------
