@@ -14,8 +14,11 @@
  *       caches c_t (width r) and one RoPE key k_rope_t (width d_r) shared by all heads.
  *
  * Conventions shared by every call:
- *   - Every data pointer is DEVICE memory owned by the caller; the library allocates nothing,
- *     keeps no state between calls (apart from a per-device SM-count cache) and never frees.
+ *   - Every data pointer is DEVICE memory owned by the caller; the library allocates nothing
+ *     and never frees. Between calls it keeps only which devices already have the attention
+ *     kernel's shared-memory limit raised (and, for mla_decode_static_workspace, each device's
+ *     address of its workspace array). mla_decode always cuts the work into 74 ranges, one
+ *     per pair of SMs of a 148-SM B200; a device with fewer SMs runs them in more than one wave.
  *   - Every call only enqueues work on `stream` (a cudaStream_t passed as void*; NULL is the
  *     legacy default stream) and returns; nothing is synchronised.
  *   - Tensors are row-major and contiguous. "dtype" tensors are float32 or bfloat16 as

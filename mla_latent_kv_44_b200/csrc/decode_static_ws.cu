@@ -51,8 +51,16 @@ extern "C" mla_status mla_decode_static_workspace(const mla_config* cfg, const v
                                                   const int32_t* seq_lens, int32_t batch,
                                                   int32_t q_per_seq, float* out_latent,
                                                   float* lse, uint32_t* dev_err, void* stream) {
-  if (!cfg || batch < 0 || q_per_seq < 1) return MLA_ERR_INVALID_ARG;
+  // The checks of mla_decode, in its order, so that both entry points return the same status
+  // for the same arguments (a configuration is valid iff it has a workspace size at batch 1);
+  // then the one check of this entry point: the workspace must fit the array.
+  if (mla_decode_workspace_size(cfg, 1, 1) == 0 || batch < 0 || q_per_seq < 1)
+    return MLA_ERR_INVALID_ARG;
   if (batch == 0) return MLA_OK;
+  if (!q || !pool || !block_table || !seq_lens || !out_latent || !dev_err)
+    return MLA_ERR_INVALID_ARG;
+  if (max_blocks < 1 || num_blocks < 1) return MLA_ERR_INVALID_ARG;
+  if ((int64_t)batch * q_per_seq > (1 << 24)) return MLA_ERR_UNSUPPORTED;
   const size_t need = mla_decode_workspace_size(cfg, batch, q_per_seq);
   if (need == 0) return MLA_ERR_INVALID_ARG;
   if (need > (size_t)MLA_STATIC_WORKSPACE_BYTES) return MLA_ERR_WORKSPACE;

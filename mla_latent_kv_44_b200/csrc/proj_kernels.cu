@@ -260,14 +260,20 @@ cudaError_t launch_output(const mla_config& c, const float* lat, const void* w_u
   dim3 grid((n + kOutTokens - 1) / kOutTokens, c.num_heads);
   if (c.dtype == MLA_BF16) {
     auto k = output_kernel<__nv_bfloat16>;
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
     return launch_pdl(k, grid, dim3(256), smem, st, lat, (const __nv_bfloat16*)w_uv,
                       (__nv_bfloat16*)o, n, c.num_heads, c.head_dim_v, c.kv_rank);
   } else {
     auto k = output_kernel<float>;
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
     return launch_pdl(k, grid, dim3(256), smem, st, lat, (const float*)w_uv, (float*)o, n,
                       c.num_heads, c.head_dim_v, c.kv_rank);
   }

@@ -81,18 +81,39 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return out
 
 
-def peaky_tolerance(Q: np.ndarray, rows: np.ndarray, w_uv: np.ndarray, kv_rank: int,
-                    scale: float, j: int, ref_o: np.ndarray, ref_lat: np.ndarray):
-    """Elementwise tolerance for outputs dominated by one cached row j (a planted needle).
+FP32_UNIT_ROUNDOFF = 2.0 ** -24
 
-    Two correct bf16 implementations may round the packed query Q or row j differently by one
-    bfloat16 ulp. Through row j's score that moves the output to first order by
-    d o / d s_j = p_j (V_j - o) times the score change, at most
-        delta = scale * sum_k (ulp(Q_k) |row_jk| + |Q_k| ulp(row_jk)).
-    The tolerance is 2e-2 of every output vector's rms plus twice that first-order change
-    (the factor covers second-order terms and the other rows' far smaller shifts).
-    Q (T, H, r + d_r) exact, rows (L, r + d_r); ref_o (T, H, d_v) and ref_lat (T, H, r) are the
-    oracle's outputs for the same inputs. Returns (tol_o, tol_lat).
+
+def bf16_rounding_ambiguous(x: np.ndarray, err: np.ndarray) -> np.ndarray:
+    """True where a value computed as x with an error of at most err may round to another
+    bfloat16 number than x itself: rounding is monotone, so that happens exactly when x - err
+    and x + err round to different numbers."""
+    from .mla_ref import round_bf16
+
+    x = np.asarray(x, dtype=np.float64)
+    err = np.broadcast_to(np.abs(np.asarray(err, dtype=np.float64)), x.shape)
+    return round_bf16(x - err) != round_bf16(x + err)
+
+
+def peaky_tolerance(Q: np.ndarray, rows: np.ndarray, w_uv: np.ndarray, kv_rank: int,
+                    scale: float, j: int, ref_o: np.ndarray, ref_lat: np.ndarray,
+                    amb_q: np.ndarray, amb_row: np.ndarray):
+    """Elementwise tolerance for outputs dominated by one cached row j (a planted needle),
+    against the oracle's bf16-query form (the exact arithmetic on the query rounded once to
+    bfloat16, which is what a bf16 boundary stores).
+
+    An implementation computes Q and row j in fp32 before rounding them to bfloat16. Where the
+    exact value lies within that computation's error bound of a rounding boundary (amb_q,
+    amb_row: see bf16_rounding_ambiguous), it may round to the neighbouring bfloat16 number.
+    Through row j's score that moves the output to first order by d o / d s_j = p_j (V_j - o)
+    times the score change, at most
+        delta = scale * (sum over ambiguous k of ulp(Q_k) |row_jk| + |Q_k| ulp(row_jk)).
+    The tolerance is 2e-2 of every output vector's rms plus twice that first-order change (the
+    factor covers second-order terms and the other rows' far smaller shifts). With no
+    ambiguous element it is the plain bf16 bar.
+    Q (T, H, r + d_r) bf16-rounded query, rows (L, r + d_r); amb_q like Q, amb_row (r + d_r);
+    ref_o (T, H, d_v) and ref_lat (T, H, r) the oracle's outputs for the same inputs.
+    Returns (tol_o, tol_lat).
     """
     from .mla_ref import _causal_lengths, softmax
 
@@ -101,10 +122,12 @@ def peaky_tolerance(Q: np.ndarray, rows: np.ndarray, w_uv: np.ndarray, kv_rank: 
     T, H, _ = Q.shape
     L = rows.shape[0]
     keep = np.arange(L)[None, :] < _causal_lengths(L, T)[:, None]
-    s = np.where(keep[:, None, :], np.einsum("thd,ld->thl", Q, rows) * scale, -np.inf)
+    s = np.where(keep[:, None, :], (Q @ rows.T) * scale, -np.inf)
     pj = softmax(s)[:, :, j]                                                   # (T, H)
     rj = rows[j]
-    delta = scale * (bf16_ulp(Q) @ np.abs(rj) + np.abs(Q) @ bf16_ulp(rj))      # (T, H)
+    uq = np.where(amb_q, bf16_ulp(Q), 0.0)
+    ur = np.where(amb_row, bf16_ulp(rj), 0.0)
+    delta = scale * (uq @ np.abs(rj) + np.abs(Q) @ ur)                         # (T, H)
     cj = rj[:kv_rank]
     Vj = np.einsum("hij,j->hi", np.asarray(w_uv, dtype=np.float64), cj)        # (H, d_v)
     sens_o = (delta * pj)[..., None] * np.abs(Vj[None] - ref_o)
@@ -113,3 +136,33 @@ def peaky_tolerance(Q: np.ndarray, rows: np.ndarray, w_uv: np.ndarray, kv_rank: 
     rms_lat = np.sqrt(np.mean(ref_lat ** 2, axis=-1, keepdims=True))
     return (BF16_SCALED_TOL * rms_o + 2.0 * sens_o,
             BF16_SCALED_TOL * rms_lat + 2.0 * sens_lat)
+
+
+def needle_ambiguity(q_nope: np.ndarray, w_uk: np.ndarray, Q_exact: np.ndarray,
+                     row_j: np.ndarray, kv_rank: int):
+    """Masks of the query and needle-row elements whose bfloat16 rounding an fp32
+    implementation may do the other way.
+
+    Q's latent part is a d_h-term fp32 sum of exact products of bf16 operands: its error is at
+    most gamma_n sum |q_i w_i| with gamma_n = n u / (1 - n u), the textbook bound of recursive
+    summation in any order, taken with u = 2^-23 (twice the fp32 unit roundoff, in case the
+    tensor core truncates its partial sums). Its RoPE part and the row's RoPE part are rotated
+    in double and rounded once (error below 2^-40 relative). The row's latent part is RMSNorm(x) * gamma in fp32: at most (r/2 + 8)
+    units in the last fp32 place of the result (the mean of r squares, a reciprocal square root
+    and two products).
+    q_nope (T, H, d_h), w_uk (H, d_h, r), Q_exact (T, H, r + d_r) unrounded, row_j (r + d_r).
+    """
+    q_nope = np.asarray(q_nope, dtype=np.float64)
+    w = np.asarray(w_uk, dtype=np.float64)
+    Q_exact = np.asarray(Q_exact, dtype=np.float64)
+    err_q = np.abs(Q_exact) * 2.0 ** -40
+    # sum_i |q_nope[t, h, i]| |w_uk[h, i, c]| for every latent column c
+    lat_err = np.einsum("thi,hic->thc", np.abs(q_nope), np.abs(w))
+    d_h = q_nope.shape[-1]
+    u = 2.0 * FP32_UNIT_ROUNDOFF
+    g = d_h * u / (1.0 - d_h * u)
+    err_q[..., :kv_rank] = g * lat_err
+    row_j = np.asarray(row_j, dtype=np.float64)
+    err_r = np.abs(row_j) * 2.0 ** -40
+    err_r[:kv_rank] = (kv_rank / 2 + 8) * FP32_UNIT_ROUNDOFF * np.abs(row_j[:kv_rank])
+    return bf16_rounding_ambiguous(Q_exact, err_q), bf16_rounding_ambiguous(row_j, err_r)

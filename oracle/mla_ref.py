@@ -268,7 +268,8 @@ def absorb_query(q_nope: np.ndarray, w_uk: np.ndarray, dtype=F64) -> np.ndarray:
     """q_lat[h] = W_UK[h]^T q_nope[h]: "DeepSeek MLA, Built From the Paper", 3 Matrix
     absorption -- q^T (W_UK c) = (W_UK^T q)^T c, so W_UK folds into the query once.
     q_nope (..., H, d_h), w_uk (H, d_h, r) -> (..., H, r)."""
-    return np.einsum("...hi,hij->...hj", np.asarray(q_nope, dtype=dtype), np.asarray(w_uk, dtype=dtype))
+    q = np.asarray(q_nope, dtype=dtype)
+    return np.matmul(q[..., None, :], np.asarray(w_uk, dtype=dtype))[..., 0, :]
 
 
 def absorbed_decode(c_kv: np.ndarray, k_rope: np.ndarray, q_nope: np.ndarray, q_rope: np.ndarray,
@@ -285,13 +286,12 @@ def absorbed_decode(c_kv: np.ndarray, k_rope: np.ndarray, q_nope: np.ndarray, q_
     L = c_kv.shape[0]
     T = q_nope.shape[0]
     q_lat = absorb_query(q_nope, w_uk, dtype)                       # (T, H, r)
-    s = (np.einsum("thj,lj->thl", q_lat, c_kv)
-         + np.einsum("thk,lk->thl", np.asarray(q_rope, dtype=dtype), k_rope)) * dtype(scale)
+    s = (q_lat @ c_kv.T + np.asarray(q_rope, dtype=dtype) @ k_rope.T) * dtype(scale)  # (T, H, L)
     keep = np.arange(L)[None, :] < _causal_lengths(L, T)[:, None]
     s = np.where(keep[:, None, :], s, -np.inf)
     p = softmax(s)
-    o_lat = np.einsum("thl,lj->thj", p, c_kv)
-    o = np.einsum("hij,thj->thi", np.asarray(w_uv, dtype=dtype), o_lat)
+    o_lat = p @ c_kv                                                # (T, H, r)
+    o = np.matmul(np.asarray(w_uv, dtype=dtype), o_lat[..., None])[..., 0]
     return DecodeOut(o, o_lat, logsumexp(s))
 
 
@@ -320,11 +320,11 @@ def latent_attention(Q: np.ndarray, rows: np.ndarray, kv_rank: int, scale: float
     """
     rows = np.asarray(rows, dtype=F64)
     L = rows.shape[0]
-    s = np.einsum("thd,ld->thl", np.asarray(Q, dtype=F64), rows) * scale
+    s = (np.asarray(Q, dtype=F64) @ rows.T) * scale                   # (T, H, L)
     keep = np.arange(L)[None, :] < _causal_lengths(L, T)[:, None]
     s = np.where(keep[:, None, :], s, -np.inf)
     p = softmax(s)
-    o_lat = np.einsum("thl,lj->thj", p, rows[:, :kv_rank])
+    o_lat = p @ rows[:, :kv_rank]
     return DecodeOut(o_lat, o_lat, logsumexp(s))
 
 
@@ -349,7 +349,8 @@ def output_ref(o_lat: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
     sum).
     o_lat (N, H, r), w_uv (H, d_v, r) -> (N, H, d_v).
     """
-    return np.einsum("hij,nhj->nhi", np.asarray(w_uv, dtype=F64), np.asarray(o_lat, dtype=F64))
+    o_lat = np.asarray(o_lat, dtype=F64)
+    return np.matmul(np.asarray(w_uv, dtype=F64), o_lat[..., None])[..., 0]
 
 
 # --------------------------------------------------------------------------------------

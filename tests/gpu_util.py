@@ -31,20 +31,30 @@ def check_sequence(state, b: int, form: str = "naive", lse_tol=None, peaky: bool
     dt = state.w.dtype
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lat)), f"seq {b}: non-finite output"
     if peaky:
-        # one needle row dominates: allow the first-order effect of a one-ulp rounding
-        # difference in the query or in that row on its score (oracle.compare.peaky_tolerance)
+        # one needle row dominates: compare with the oracle's bf16-query form (the exact
+        # arithmetic on the query rounded once to bfloat16, as the boundary stores it) under
+        # the plain bar plus the first-order effect of the query and needle-row elements whose
+        # rounding an fp32 computation may do the other way (oracle.compare.peaky_tolerance)
         w = state.w
         ckv, kr, qn, qr = state.host_draws[b]
         n = ckv.shape[0]
+        j = state.needle_rows[b]
+        exp = ref.decode_sequence_bf16_query(ckv, kr, qn, qr, state.w_uk_host, state.w_uv_host,
+                                             state.gamma_host, w.softmax_scale, w.rms_eps,
+                                             w.rope_base)
         rows = ref.cache_rows(ckv, kr, state.gamma_host, np.arange(n), w.rms_eps, w.rope_base,
                               True)
-        Q = ref.absorb_ref(qn, qr, np.arange(n - w.new_tokens, n), state.w_uk_host, w.rope_base)
-        tol_o, tol_l = compare.peaky_tolerance(Q, rows, state.w_uv_host, w.kv_rank,
-                                               w.softmax_scale, state.needle_rows[b], exp.o,
-                                               exp.o_lat)
+        Qx = ref.absorb_ref(qn, qr, np.arange(n - w.new_tokens, n), state.w_uk_host, w.rope_base)
+        amb_q, amb_r = compare.needle_ambiguity(qn, state.w_uk_host, Qx, rows[j], w.kv_rank)
+        tol_o, tol_l = compare.peaky_tolerance(ref.round_bf16(Qx), rows, state.w_uv_host,
+                                               w.kv_rank, w.softmax_scale, j, exp.o, exp.o_lat,
+                                               amb_q, amb_r)
+        widen = needle_widening(tol_o, exp.o)
+        assert widen <= NEEDLE_MAX_WIDENING, f"seq {b}: needle tolerance {widen:.2f}x the plain bar"
         assert np.all(np.abs(o - exp.o) <= tol_o), f"seq {b}: output outside the needle tolerance"
         assert np.all(np.abs(lat - exp.o_lat) <= tol_l), f"seq {b}: latent outside the needle tolerance"
-        e_o = e_l = 0.0
+        e_o = float(np.max(np.abs(o - exp.o) / (compare.BF16_SCALED_TOL * _vec_rms(exp.o))))
+        e_l = float(np.max(np.abs(lat - exp.o_lat) / (compare.BF16_SCALED_TOL * _vec_rms(exp.o_lat))))
     else:
         ok_o, e_o = compare.within(o, exp.o, dt)
         ok_l, e_l = compare.within(lat, exp.o_lat, dt)
@@ -55,6 +65,20 @@ def check_sequence(state, b: int, form: str = "naive", lse_tol=None, peaky: bool
     if not peaky:
         assert e_lse <= tol, f"seq {b}: lse error {e_lse}"
     return e_o, e_l, e_lse
+
+
+# The needle tolerance may exceed the plain 2e-2 bar only by the first-order effect of
+# ambiguous roundings; on the needle inputs of the tests that is at most about 2.2x the bar.
+NEEDLE_MAX_WIDENING = 4.0
+
+
+def _vec_rms(x):
+    return np.sqrt(np.mean(np.asarray(x, dtype=np.float64) ** 2, axis=-1, keepdims=True))
+
+
+def needle_widening(tol, ref_out) -> float:
+    """max over elements of the needle tolerance over the plain bar (2e-2 of its vector's rms)."""
+    return float(np.max(tol / (compare.BF16_SCALED_TOL * _vec_rms(ref_out))))
 
 
 def dev_err(state) -> int:

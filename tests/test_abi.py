@@ -116,3 +116,37 @@ def test_product_package_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in re.findall(r"^\s*(?:from|import)\s+(\w+)", text, re.M), f
+
+
+def _decode_both(mla, c, batch, q_per_seq, **ptrs):
+    """Status of mla_decode (with a large enough workspace) and of mla_decode_static_workspace
+    for the same arguments; every case here fails or succeeds before any CUDA call."""
+    p = dict(q=256, pool=256, table=256, lens=256, out=256, err=256)
+    p.update(ptrs)
+    ws = mla.lib.mla_decode_workspace_size(ctypes.byref(c), max(batch, 1), max(q_per_seq, 1))
+    a = mla.lib.mla_decode(ctypes.byref(c), p["q"], p["pool"], p["table"], 4, 4, p["lens"], batch,
+                           q_per_seq, 256, max(ws, 1), p["out"], None, p["err"], None)
+    b = mla.lib.mla_decode_static_workspace(ctypes.byref(c), p["q"], p["pool"], p["table"], 4, 4,
+                                            p["lens"], batch, q_per_seq, p["out"], None, p["err"],
+                                            None)
+    return a, b
+
+
+def test_static_workspace_entry_point_returns_mla_decodes_statuses(mla):
+    good = _cfg(mla)
+    bad = _cfg(mla, kv_rank=48)
+    # an invalid configuration is reported even when there is no work
+    assert _decode_both(mla, bad, 0, 1) == (mla.MLA_ERR_INVALID_ARG, mla.MLA_ERR_INVALID_ARG)
+    assert _decode_both(mla, good, 0, 1) == (mla.MLA_OK, mla.MLA_OK)
+    assert _decode_both(mla, good, -1, 1) == (mla.MLA_ERR_INVALID_ARG, mla.MLA_ERR_INVALID_ARG)
+    assert _decode_both(mla, good, 2, 0) == (mla.MLA_ERR_INVALID_ARG, mla.MLA_ERR_INVALID_ARG)
+    assert _decode_both(mla, good, 2, 1, q=None) == (mla.MLA_ERR_INVALID_ARG,
+                                                      mla.MLA_ERR_INVALID_ARG)
+    # more (sequence, token) pairs than the schedule supports: unsupported, not invalid
+    assert _decode_both(mla, good, 1 << 22, 8) == (mla.MLA_ERR_UNSUPPORTED, mla.MLA_ERR_UNSUPPORTED)
+    # a workspace larger than the library's array is the static entry point's own error
+    big = 100000
+    assert mla.lib.mla_decode_workspace_size(ctypes.byref(good), big, 1) > mla.STATIC_WORKSPACE_BYTES
+    st = mla.lib.mla_decode_static_workspace(ctypes.byref(good), 256, 256, 256, 4, 4, 256, big, 1,
+                                             256, None, 256, None)
+    assert st == mla.MLA_ERR_WORKSPACE

@@ -76,21 +76,37 @@ def test_needle_peaky_attention(mla, name):
 # Whole step, full-size workloads: every sequence decoded, sampled sequences checked
 # ----------------------------------------------------------------------------------------
 
+def _split_sequences(rows, T):
+    """Sequences with a row group that the planner splits across work ranges (from the split
+    rule restated on the host in tests/test_plan.py)."""
+    from tests.test_plan import expected_plan
+
+    plan = expected_plan([int(x) for x in rows], T, int(max(rows)))
+    return sorted({bt // T for bt, n in enumerate(plan["bt_nseg"]) if n >= 2})
+
+
 @pytest.mark.parametrize("name", ["dsv2", "ragged", "mtp"])
 def test_full_step_large(mla, name):
+    """Full-size DeepSeek-V2-shaped steps. C3 (64 sequences) and C5 (32): every sequence is
+    checked; C4 (128 ragged sequences): every sequence with a split row group (each of the
+    planner's range boundaries inside a sequence) and a fixed sample of 16 others. The two
+    shortest checked sequences go against the naive form, the rest against the absorbed
+    float64 cross-form (the naive form costs about 0.3 TFLOP per 8k-row sequence)."""
     from mla_latent_kv_44_b200.step import DecodeState
 
     w = mi.WORKLOADS[name]
-    samples = mi.sample_sequences(w, 3)
-    st = DecodeState(w, sequences=samples)
+    rows = mi.total_rows(w, 0)
+    if name == "ragged":
+        seqs = sorted(set(_split_sequences(rows, w.new_tokens)) | set(mi.sample_sequences(w, 16)))
+        assert len(seqs) >= 16
+    else:
+        seqs = list(range(w.batch))
+    st = DecodeState(w, sequences=seqs)
     st.step()
     assert dev_err(st) == 0
-    rows = st.rows
-    shortest = min(samples, key=lambda b: rows[b])
-    check_sequence(st, shortest, "naive")
-    for b in samples:
-        if b != shortest:
-            check_sequence(st, b, "absorbed")
+    naive = sorted(seqs, key=lambda b: rows[b])[:2]
+    for b in seqs:
+        check_sequence(st, b, "naive" if b in naive else "absorbed")
     # every output row is finite (no sentinel rows leaked into any sequence)
     assert torch.isfinite(st.out_latent).all() and torch.isfinite(st.o.float()).all()
 
