@@ -109,8 +109,8 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------------------
-# SM clocks and clock-event reasons, read through NVML every 10 ms by a host thread while the
-# timed region runs (read-only queries; nothing is set). nvidia-smi is the fallback.
+# SM clocks and clock-event reasons, read through NVML every 2 ms by a host thread over the
+# warm-up and the timed region (read-only queries; nothing is set). nvidia-smi is the fallback.
 # ---------------------------------------------------------------------------------------
 class ClockSampler:
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
@@ -122,7 +122,7 @@ class ClockSampler:
                   "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                   "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, uuid: str, index: int, period_s: float = 0.01):
+    def __init__(self, uuid: str, index: int, period_s: float = 0.002):
         self.uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         self.index = index
         self.period = period_s
@@ -196,9 +196,9 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self._proc.kill()
 
-    def summary(self, t0, t1):
+    def summary(self, t0, t1, label="timed region"):
         rows = [s for s in self.samples if t0 <= s[0] <= t1]
-        window = "timed region"
+        window = label
         if not rows and self.samples:
             mid = 0.5 * (t0 + t1)
             rows = sorted(self.samples, key=lambda s: abs(s[0] - mid))[:3]
@@ -248,9 +248,25 @@ def blas_threads():
         return os.cpu_count()
 
 
+def _absorbed_run(w, inputs):
+    from oracle import mla_ref
+
+    ckv, kr, qn, qr, wuk, wuv, gamma = inputs
+    return mla_ref.decode_sequence_from_raw(ckv, kr, qn, qr, wuk, wuv, gamma, w.softmax_scale,
+                                            w.rms_eps, w.rope_base, store_bf16=(w.dtype == "bf16"),
+                                            form="absorbed")
+
+
 def cpu_baseline(w, budget_s: float = 15.0):
-    """Naive float64 oracle over whole sequences of the workload (all heads), one after another,
-    until about ``budget_s`` seconds of oracle time; input generation is not timed."""
+    """The float64 oracle on the host's cores, three ways (input generation is not timed):
+
+    * the naive form (K and V rebuilt per head), all heads, whole sequences one after another
+      until about ``budget_s`` seconds -- the line's value;
+    * the same form on one BLAS thread, on a subset of the heads of sequence 0 (scaled to all
+      heads);
+    * the absorbed float64 form over the whole batch (every sequence, all heads), or as many
+      sequences as fit in 3 * budget_s seconds, scaled to the batch and marked extrapolated.
+    """
     n, spent, rows = 0, 0.0, 0
     while n < w.batch and spent < budget_s:
         inp = oracle_sample(w, w.num_heads, seq=n)
@@ -259,12 +275,41 @@ def cpu_baseline(w, budget_s: float = 15.0):
         spent += time.perf_counter() - t0
         rows += int(inp[0].shape[0])
         n += 1
-    return {"value": n * w.new_tokens / spent, "unit": "tokens/s", "cores": blas_threads(),
+    line = {"value": n * w.new_tokens / spent, "unit": "tokens/s", "cores": blas_threads(),
             "kind": "oracle",
             "sample": (f"naive float64 oracle (K and V rebuilt per head, all {w.num_heads} heads): "
                        f"sequences 0-{n - 1} of {w.name} ({rows} cached rows in all), "
                        f"{spent:.1f} s of oracle time on the host's cores; value = query tokens "
                        f"per second")}
+    try:
+        from threadpoolctl import threadpool_limits
+
+        heads = max(1, w.num_heads // 16)
+        inp = oracle_sample(w, heads, seq=0)
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            oracle_run(w, inp)
+            dt1 = time.perf_counter() - t0
+        line["naive_one_thread"] = {
+            "value": w.new_tokens / (dt1 * w.num_heads / heads), "unit": "tokens/s", "cores": 1,
+            "sample": f"naive float64 oracle on one BLAS thread, {heads} of {w.num_heads} heads of "
+                      f"sequence 0 ({dt1:.1f} s), scaled to all heads"}
+    except ImportError:
+        line["naive_one_thread"] = None
+    n2, spent2 = 0, 0.0
+    while n2 < w.batch and spent2 < 3 * budget_s:
+        inp = oracle_sample(w, w.num_heads, seq=n2)
+        t0 = time.perf_counter()
+        _absorbed_run(w, inp)
+        spent2 += time.perf_counter() - t0
+        n2 += 1
+    line["absorbed_f64_batch"] = {
+        "value": n2 * w.new_tokens / spent2, "unit": "tokens/s", "cores": blas_threads(),
+        "sequences": n2, "of": w.batch, "extrapolated": n2 < w.batch,
+        "seconds_per_batch": spent2 * w.batch / n2,
+        "sample": f"absorbed float64 oracle (W_UK folded into the query), {n2} of {w.batch} "
+                  f"sequences, all heads, {spent2:.1f} s on the host's cores"}
+    return line
 
 
 def run_reference(args, w):
@@ -369,6 +414,13 @@ def run_ours(args, w):
         if world > 1:
             dist.barrier()
 
+    props = torch.cuda.get_device_properties(dev)
+    clock = ClockSampler(str(getattr(props, "uuid", "")), local)
+    if rank == 0:
+        clock.start()
+    barrier()
+    t_warm0 = time.time()
+
     # ---- warm-up ----
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
@@ -377,37 +429,23 @@ def run_ours(args, w):
     if int(st.dev_err.item()) != 0:
         raise RuntimeError(f"device error bits {int(st.dev_err.item())}")
 
-    # ---- timed region: K steps. Events on the launching stream bracket the attention kernel
-    # (for the roofline) and each step; the other kernels follow one another with programmatic
-    # dependent launch, which an event between them would break.
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # ---- timed region: K steps, one event before and one after. Inside, the kernels follow one
+    # another with programmatic dependent launch (each starts its set-up while the previous one
+    # drains), which an event between them would break.
+    ev_start = torch.cuda.Event(enable_timing=True)
     ev_end = torch.cuda.Event(enable_timing=True)
-    props = torch.cuda.get_device_properties(dev)
-    clock = ClockSampler(str(getattr(props, "uuid", "")), local)
-    if rank == 0:
-        clock.start()
-    barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
     with torch.cuda.stream(stream):
-        for k in range(args.steps):
-            e = ev[k]
-            e[0].record(stream)
-            st.absorb(stream)
-            st.append(stream)
-            st.attend(stream, mla.STAGE_PLAN)
-            e[1].record(stream)
-            st.attend(stream, mla.STAGE_ATTEND)
-            e[2].record(stream)
-            st.attend(stream, mla.STAGE_COMBINE)
-            st.project(stream)
+        ev_start.record(stream)
+        for _ in range(args.steps):
+            st.step(stream)
         ev_end.record(stream)
     stream.synchronize()
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
     barrier()
-    elapsed_ms = ev[0][0].elapsed_time(ev_end)
-    attend_only_ms = sum(ev[k][1].elapsed_time(ev[k][2]) for k in range(args.steps)) / args.steps
+    elapsed_ms = ev_start.elapsed_time(ev_end)
     if int(st.dev_err.item()) != 0:
         raise RuntimeError(f"device error bits {int(st.dev_err.item())}")
 
@@ -428,6 +466,9 @@ def run_ours(args, w):
     stream.synchronize()
     stage_ms = {n: sum(evd[k][i].elapsed_time(evd[k][i + 1]) for k in range(n_detail)) / n_detail
                 for i, n in enumerate(names)}
+    # the attention kernel's own duration (the roofline's denominator): from this run, where an
+    # event on its stream brackets every launch
+    attend_only_ms = stage_ms["attend"]
 
     # ---- e2e through host buffers: every step uploads its inputs from pinned host memory (one
     # packed copy) and reads its output o back. Steps are pipelined over two input and two
@@ -505,7 +546,7 @@ def run_ours(args, w):
                                                    world, dev)
     if rank == 0:
         clock.stop()
-    clocks = clock.summary(t_wall0, t_wall1) if rank == 0 else None
+    clocks = clock.summary(t_warm0, t_wall1, "warm-up and timed steps") if rank == 0 else None
     del st
     if world > 1:
         dist.destroy_process_group()

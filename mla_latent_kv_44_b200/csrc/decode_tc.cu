@@ -89,7 +89,7 @@ constexpr int kDataBytes = kS_End > kV_End ? kS_End : kV_End;
 // segments of the work range, staged once per CTA (longer ranges read the rest from global)
 constexpr int kSegCache = 64;
 constexpr int kSegOff = kDataBytes;
-constexpr int kSegBytes = kSegCache * 24;
+constexpr int kSegBytes = kSegCache * 28;
 
 enum Bar {
   // score CTA
@@ -177,14 +177,15 @@ __device__ void drain_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
   if (!done && (threadIdx.x & 31) == 0) set_error(err, MLA_DEV_WAIT_TIMEOUT);
 }
 
-// A segment of the work range with the fields of its row group.
+// A segment of the work range with the fields of its row group (b: its sequence).
 struct SegInfo {
-  int bt, chunk_lo, chunk_hi, slot, chunk0, len;
+  int bt, chunk_lo, chunk_hi, slot, chunk0, len, b;
 };
 
 __device__ __forceinline__ SegInfo load_segment(const DecodeParams& p, int s) {
   const Segment sg = p.segments[s];
-  return SegInfo{sg.bt, sg.chunk_lo, sg.chunk_hi, sg.slot, p.bt_chunk0[sg.bt], p.bt_len[sg.bt]};
+  return SegInfo{sg.bt, sg.chunk_lo, sg.chunk_hi, sg.slot, p.bt_chunk0[sg.bt], p.bt_len[sg.bt],
+                 sg.bt / p.T};
 }
 
 // One score tile: up to two consecutive cache blocks of one segment.
@@ -211,7 +212,7 @@ struct TileWalk {
       if (c < cur.chunk_lo) c = cur.chunk_lo;
       if (c < cur.chunk_hi) {
         tl.bt = cur.bt;
-        tl.b = cur.bt / p->T;
+        tl.b = cur.b;
         tl.local0 = c - cur.chunk0;
         tl.nb = min(kTileBlocks, cur.chunk_hi - c);
         tl.ntok = min(tl.nb * kRows, cur.len - tl.local0 * kRows);
@@ -403,7 +404,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
     // still queued).
     if (lane == 0) {
       int kt = 0, t = 0, seg_i = 0;
-      bool ok = true;
+      bool ok = true, next_ready = false;
       while (ok && walk.next(tl)) {
         if (tl.first) {
           // the previous segment's S products have finished reading Q from TMEM
@@ -441,7 +442,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
         // next stage's barrier is tested (without blocking) between a stage's MMAs, while two of
         // them are queued: a barrier read takes longer than one MMA, and a stage already seen
         // complete needs no wait at its start.
-        bool next_ready = false;
+        if (tl.first) next_ready = false;
 #pragma unroll 1
         for (int k = 0; k < 9; ++k, ++kt) {
           const int stage = kt % kKStages;
@@ -461,9 +462,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 4; ++i) {
               mma_ss(d, sdesc(s_base + kS_QRope + 32 * i, 16, 1024, 2),
                      sdesc(kb + 32 * i, 16, 1024, 2), id, 1u);
+              // the next tile's first stage (of the same segment; a new segment's first
+              // stages carry its query and are waited for as usual)
+              if (i == 1) next_ready = mbar_test(bar(kKFull + nkt % kKStages), (nkt / kKStages) & 1);
+            }
           }
           tc_commit(bar(kKEmpty + stage));
         }
