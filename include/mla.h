@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 2
+#define MLA_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define MLA_API __attribute__((visibility("default")))
@@ -206,6 +206,36 @@ MLA_API mla_status mla_decode_static_workspace(const mla_config* cfg, const void
  */
 MLA_API mla_status mla_output(const mla_config* cfg, const float* out_latent, const void* w_uv, void* o,
                       int32_t n_tokens, uint32_t* dev_err, void* stream);
+
+/*
+ * mla_decode_step -- one whole decode step: exactly mla_absorb_query, mla_append_latent,
+ * mla_decode and mla_output called in that order with these arguments (the sources of each are
+ * cited above), for n = batch * q_per_seq new tokens, token k = b * q_per_seq + t being query
+ * token t of sequence b:
+ *   mla_absorb_query(cfg, q_nope, q_rope, pos, w_uk, q_work, n)
+ *   mla_append_latent(cfg, ckv_raw, krope_raw, gamma, seq_idx, pos, block_table, batch,
+ *                     max_blocks, pool, num_blocks, n)
+ *   mla_decode(cfg, q_work, pool, block_table, max_blocks, num_blocks, seq_lens, batch,
+ *              q_per_seq, workspace, workspace_bytes, out_latent, lse)
+ *   mla_output(cfg, out_latent, w_uv, o, n)
+ * so pos and seq_idx are the new tokens' positions and sequences, and seq_lens already counts
+ * the new rows. q_work (n, H, r + d_r) dtype receives the absorbed query. The results (q_work,
+ * the pool's new rows, out_latent, lse, o, *dev_err) are bit for bit those of the four calls.
+ * Every argument is validated as the four calls validate theirs before anything is enqueued
+ * (the same status codes). Where the tensor-core kernels apply to every stage (bf16, the
+ * attention kernel's shape, 16-byte aligned operands) the step takes four launches instead of
+ * six: the absorbed query, the append and the decode planner run as parts of one grid (they do
+ * not depend on one another), followed by the attention, the combine and the output
+ * projection; otherwise the four calls' own kernels run in order.
+ */
+MLA_API mla_status mla_decode_step(const mla_config* cfg, const void* q_nope, const void* q_rope,
+                                   const void* w_uk, const void* ckv_raw, const void* krope_raw,
+                                   const float* gamma, const int32_t* seq_idx, const int32_t* pos,
+                                   const int32_t* block_table, int32_t max_blocks, void* pool,
+                                   int32_t num_blocks, const int32_t* seq_lens, int32_t batch,
+                                   int32_t q_per_seq, void* q_work, void* workspace,
+                                   size_t workspace_bytes, float* out_latent, float* lse,
+                                   const void* w_uv, void* o, uint32_t* dev_err, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 MLA_API const char* mla_status_string(mla_status status);

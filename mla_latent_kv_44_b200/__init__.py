@@ -60,6 +60,9 @@ def _load():
         "mla_output": (_c_i32, [P, _vp, _vp, _vp, _c_i32, _vp, _vp]),
         "mla_decode_static_workspace": (_c_i32, [P, _vp, _vp, _vp, _c_i32, _c_i32, _vp, _c_i32,
                                                  _c_i32, _vp, _vp, _vp, _vp]),
+        "mla_decode_step": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _vp,
+                                     _c_i32, _vp, _c_i32, _c_i32, _vp, _vp, _sz, _vp, _vp, _vp,
+                                     _vp, _vp, _vp]),
         "mla_status_string": (ctypes.c_char_p, [_c_i32]),
         "mla_abi_version": (_c_i32, []),
     }
@@ -187,6 +190,22 @@ def decode_static_workspace(cfg: Config, q, pool, block_table, seq_lens, q_per_s
                                            int(seq_lens.shape[0]), q_per_seq, _ptr(out_latent),
                                            _ptr(lse), _ptr(dev_err), _stream(stream)),
            "mla_decode_static_workspace")
+
+
+def decode_step(cfg: Config, q_nope, q_rope, w_uk, ckv_raw, krope_raw, gamma, seq_idx, pos,
+                block_table, pool, seq_lens, q_per_seq: int, q_work, workspace, out_latent, lse,
+                w_uv, o, dev_err, stream=None):
+    """mla_decode_step: absorb, append, decode and output of one step in one call (see
+    include/mla.h); batch = seq_lens.shape[0]."""
+    c = cfg.c()
+    _check(lib.mla_decode_step(ctypes.byref(c), _ptr(q_nope), _ptr(q_rope), _ptr(w_uk),
+                               _ptr(ckv_raw), _ptr(krope_raw), _ptr(gamma), _ptr(seq_idx), _ptr(pos),
+                               _ptr(block_table), int(block_table.shape[1]), _ptr(pool),
+                               int(pool.shape[0]), _ptr(seq_lens), int(seq_lens.shape[0]),
+                               q_per_seq, _ptr(q_work), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _ptr(out_latent),
+                               _ptr(lse), _ptr(w_uv), _ptr(o), _ptr(dev_err), _stream(stream)),
+           "mla_decode_step")
 
 
 def output(cfg: Config, out_latent, w_uv, o, stream=None, dev_err=None):

@@ -163,5 +163,12 @@ cudaError_t launch_absorb_tc(const mla_config& c, const void* q_nope, const void
                              uint32_t* err, cudaStream_t st);
 cudaError_t launch_output_tc(const mla_config& c, const float* lat, const void* w_uv, void* o,
                              int n, uint32_t* err, cudaStream_t st);
+// The fused step's first launch: absorb tiles, append rows and the planner as CTA roles of one
+// grid (bf16, shapes where absorb_tc_supported and append's vector path hold).
+cudaError_t launch_step_prep(const mla_config& c, const void* q_nope, const void* q_rope,
+                             const int32_t* pos, const void* w_uk, void* q_out, int n,
+                             const void* ckv, const void* kr, const float* gamma,
+                             const int32_t* seq, const DecodeParams& p, void* pool,
+                             cudaStream_t st);
 
 }  // namespace mla

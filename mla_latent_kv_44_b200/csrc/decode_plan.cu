@@ -7,154 +7,15 @@
 // straight to the output; a row group crossed by range boundaries becomes several segments
 // whose softmax-normalised partial results (with their log-sum-exp) are merged by the combine
 // kernel. Integer work only: the schedule is a pure function of seq_lens.
-#include "common.cuh"
+#include "plan_body.cuh"
 
 namespace mla {
 
-// Number of range starts strictly below chunk x: #{q in [0,R) : floor(q*C/R) < x}.
-__device__ __forceinline__ int starts_below(int64_t x, int64_t R, int64_t C) {
-  if (x <= 0 || C <= 0) return 0;
-  const int64_t v = (x * R + C - 1) / C;
-  return (int)(v < R ? v : R);
-}
-
-__device__ __forceinline__ int range_start(int64_t q, int64_t R, int64_t C) {
-  return (int)((q * C) / R);
-}
-
 constexpr int kPlanThreads = 1024;
 
-// Inclusive block scan of two ints over kPlanThreads threads: shuffle scans inside each warp,
-// then one warp scans the 32 warp totals. s_a / s_b hold at least 32 ints.
-__device__ void block_scan2(int* s_a, int* s_b, int& a, int& b) {
-  static_assert(kPlanThreads == 32 * 32, "one warp scans the warp totals");
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int va = __shfl_up_sync(0xffffffffu, a, o), vb = __shfl_up_sync(0xffffffffu, b, o);
-    if (lane >= o) {
-      a += va;
-      b += vb;
-    }
-  }
-  if (lane == 31) {
-    s_a[warp] = a;
-    s_b[warp] = b;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    int wa = s_a[lane], wb = s_b[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int va = __shfl_up_sync(0xffffffffu, wa, o), vb = __shfl_up_sync(0xffffffffu, wb, o);
-      if (lane >= o) {
-        wa += va;
-        wb += vb;
-      }
-    }
-    s_a[lane] = wa;
-    s_b[lane] = wb;
-  }
-  __syncthreads();
-  if (warp > 0) {
-    a += s_a[warp - 1];
-    b += s_b[warp - 1];
-  }
-  __syncthreads();  // s_a / s_b are reused by the next scan
-}
-
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(DecodeParams p) {
-  __shared__ int s_a[32], s_b[32];
-  __shared__ int s_carry_a, s_carry_b;
-  const int tid = threadIdx.x;
-  const int64_t cap = (int64_t)p.max_blocks * p.bs;
-  wait_prior_grid();
-
-  // Pass 1: attended lengths, chunk counts, exclusive prefix of chunk counts. With at most
-  // kPlanThreads row groups (one pass), pass 2 takes them from registers.
-  int my_len = 0, my_chunk0 = 0;
-  if (tid == 0) s_carry_a = 0;
-  __syncthreads();
-  for (int base = 0; base < p.BT; base += kPlanThreads) {
-    const int bt = base + tid;
-    int nch = 0;
-    if (bt < p.BT) {
-      const int b = bt / p.T, t = bt - b * p.T;
-      const int sl = p.seq_lens[b];
-      int len = 0;
-      if (sl < p.T || (int64_t)sl > cap) {
-        if (t == 0) set_error(p.err, MLA_DEV_BAD_LENGTH);
-      } else {
-        len = sl - p.T + 1 + t;
-      }
-      nch = (len + kChunk - 1) / kChunk;
-      p.bt_len[bt] = len;
-      my_len = len;
-    }
-    int inc = nch, dummy = 0;
-    block_scan2(s_a, s_b, inc, dummy);
-    if (bt < p.BT) {
-      my_chunk0 = s_carry_a + inc - nch;
-      p.bt_chunk0[bt] = my_chunk0;
-    }
-    __syncthreads();
-    if (tid == kPlanThreads - 1) s_carry_a += inc;
-    __syncthreads();
-  }
-  const int C = s_carry_a;
-  const int R = C < kRanges ? C : kRanges;
-  __syncthreads();
-
-  // Pass 2: segments per row group, their global indices and partial-result slots.
-  if (tid == 0) { s_carry_a = 0; s_carry_b = 0; }
-  __syncthreads();
-  for (int base = 0; base < p.BT; base += kPlanThreads) {
-    const int bt = base + tid;
-    int nseg = 0, nslot = 0, x = 0, e = 0;
-    if (bt < p.BT) {
-      const bool one_pass = p.BT <= kPlanThreads;
-      const int len = one_pass ? my_len : p.bt_len[bt];
-      const int nch = (len + kChunk - 1) / kChunk;
-      x = one_pass ? my_chunk0 : p.bt_chunk0[bt];
-      e = x + nch;
-      if (nch > 0) nseg = 1 + starts_below(e, R, C) - starts_below(x + 1, R, C);
-      nslot = nseg >= 2 ? nseg : 0;
-    }
-    int inc_seg = nseg, inc_slot = nslot;
-    block_scan2(s_a, s_b, inc_seg, inc_slot);
-    if (bt < p.BT) {
-      const int first = s_carry_a + inc_seg - nseg;
-      const int slot0 = s_carry_b + inc_slot - nslot;
-      p.bt_slot0[bt] = nseg >= 2 ? slot0 : -1;
-      p.bt_nseg[bt] = nseg;
-      // cut points of this row group: x, the range starts strictly inside (x, e), e
-      int q = starts_below(x + 1, R, C);  // first range starting after x
-      int lo = x;
-      for (int k = 0; k < nseg; ++k) {
-        const int hi = (k == nseg - 1) ? e : range_start(q, R, C);
-        Segment sg;
-        sg.bt = bt;
-        sg.chunk_lo = lo;
-        sg.chunk_hi = hi;
-        sg.slot = nseg >= 2 ? slot0 + k : -1;
-        p.segments[first + k] = sg;
-        // a range starting exactly here begins with this segment
-        const int qs = starts_below(lo + 1, R, C) - 1;  // range containing chunk lo
-        if (qs >= 0 && range_start(qs, R, C) == lo) p.range_begin[qs] = first + k;
-        lo = hi;
-        ++q;
-      }
-    }
-    __syncthreads();
-    if (tid == kPlanThreads - 1) { s_carry_a += inc_seg; s_carry_b += inc_slot; }
-    __syncthreads();
-  }
-  if (tid == 0) {
-    p.header[0] = s_carry_a;  // segments
-    p.header[1] = R;          // ranges in use
-    p.header[2] = C;          // chunks
-    p.range_begin[R] = s_carry_a;
-  }
+  __shared__ int s_a[32], s_b[32], s_carry[2];
+  plan_body<kPlanThreads>(p, s_a, s_b, s_carry);
 }
 
 cudaError_t launch_plan(const DecodeParams& p, cudaStream_t st) {
@@ -182,21 +43,12 @@ __global__ void __launch_bounds__(kCombineHeads * 32) combine_kernel(DecodeParam
   if (h >= p.H) return;
   float4* dst = (float4*)(p.out + ((size_t)bt * p.H + h) * p.r);
   const int r4 = p.r / 4;
-  float mx = -INFINITY;
-  for (int k = lane; k < nseg; k += 32) mx = fmaxf(mx, p.part_lse[(size_t)(slot0 + k) * p.H + h]);
-  mx = warp_max(mx);
-  if (nseg == 0 || mx == -INFINITY) {  // no rows (bad length, or every block rejected)
+  const float L = merge_weights(p, slot0, nseg, h, s_w[warp]);
+  if (L == -INFINITY) {  // no rows (bad length, or every block rejected)
     for (int d = lane; d < r4; d += 32) dst[d] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (lane == 0 && p.lse) p.lse[(size_t)bt * p.H + h] = -INFINITY;
     return;
   }
-  float z = 0.f;
-  for (int k = lane; k < nseg; k += 32) z += expf(p.part_lse[(size_t)(slot0 + k) * p.H + h] - mx);
-  z = warp_sum(z);
-  const float L = mx + logf(z);
-  for (int k = lane; k < nseg; k += 32)
-    s_w[warp][k] = expf(p.part_lse[(size_t)(slot0 + k) * p.H + h] - L);
-  __syncwarp();
   // a lane holds up to four float4 of the row at once (r = 512 in one pass), so every partial's
   // loads for the whole row are in flight together
   for (int d0 = lane; d0 < r4; d0 += 128) {

@@ -30,6 +30,44 @@ mla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+DecodeParams make_params(const mla_config* cfg, const void* q, const void* pool,
+                         const int32_t* block_table, int32_t max_blocks, int32_t num_blocks,
+                         const int32_t* seq_lens, int32_t batch, int32_t q_per_seq,
+                         void* workspace, float* out_latent, float* lse, uint32_t* dev_err) {
+  const int bt = batch * q_per_seq;
+  const WorkspaceLayout L = workspace_layout(cfg->num_heads, cfg->kv_rank, bt);
+  char* ws = static_cast<char*>(workspace);
+  DecodeParams p;
+  p.q = q;
+  p.pool = pool;
+  p.table = block_table;
+  p.seq_lens = seq_lens;
+  p.out = out_latent;
+  p.lse = lse;
+  p.err = dev_err;
+  p.header = reinterpret_cast<int32_t*>(ws + L.header);
+  p.range_begin = reinterpret_cast<int32_t*>(ws + L.range_begin);
+  p.segments = reinterpret_cast<Segment*>(ws + L.segments);
+  p.bt_slot0 = reinterpret_cast<int32_t*>(ws + L.bt_slot0);
+  p.bt_nseg = reinterpret_cast<int32_t*>(ws + L.bt_nseg);
+  p.bt_len = reinterpret_cast<int32_t*>(ws + L.bt_len);
+  p.bt_chunk0 = reinterpret_cast<int32_t*>(ws + L.bt_chunk0);
+  p.part_lse = reinterpret_cast<float*>(ws + L.part_lse);
+  p.part_o = reinterpret_cast<float*>(ws + L.part_o);
+  p.H = cfg->num_heads;
+  p.r = cfg->kv_rank;
+  p.dr = cfg->rope_dim;
+  p.D = cfg->kv_rank + cfg->rope_dim;
+  p.bs = cfg->block_size;
+  p.max_blocks = max_blocks;
+  p.num_blocks = num_blocks;
+  p.batch = batch;
+  p.T = q_per_seq;
+  p.BT = bt;
+  p.scale = cfg->softmax_scale;
+  return p;
+}
+
 }  // namespace
 
 extern "C" {
@@ -119,36 +157,8 @@ mla_status mla_decode_stages(const mla_config* cfg, int32_t stages, const void* 
     default: use_tc = tc_supported(*cfg); break;
   }
 
-  const WorkspaceLayout L = workspace_layout(cfg->num_heads, cfg->kv_rank, (int)bt);
-  char* ws = static_cast<char*>(workspace);
-  DecodeParams p;
-  p.q = q;
-  p.pool = pool;
-  p.table = block_table;
-  p.seq_lens = seq_lens;
-  p.out = out_latent;
-  p.lse = lse;
-  p.err = dev_err;
-  p.header = reinterpret_cast<int32_t*>(ws + L.header);
-  p.range_begin = reinterpret_cast<int32_t*>(ws + L.range_begin);
-  p.segments = reinterpret_cast<Segment*>(ws + L.segments);
-  p.bt_slot0 = reinterpret_cast<int32_t*>(ws + L.bt_slot0);
-  p.bt_nseg = reinterpret_cast<int32_t*>(ws + L.bt_nseg);
-  p.bt_len = reinterpret_cast<int32_t*>(ws + L.bt_len);
-  p.bt_chunk0 = reinterpret_cast<int32_t*>(ws + L.bt_chunk0);
-  p.part_lse = reinterpret_cast<float*>(ws + L.part_lse);
-  p.part_o = reinterpret_cast<float*>(ws + L.part_o);
-  p.H = cfg->num_heads;
-  p.r = cfg->kv_rank;
-  p.dr = cfg->rope_dim;
-  p.D = cfg->kv_rank + cfg->rope_dim;
-  p.bs = cfg->block_size;
-  p.max_blocks = max_blocks;
-  p.num_blocks = num_blocks;
-  p.batch = batch;
-  p.T = q_per_seq;
-  p.BT = (int)bt;
-  p.scale = cfg->softmax_scale;
+  const DecodeParams p = make_params(cfg, q, pool, block_table, max_blocks, num_blocks, seq_lens,
+                                     batch, q_per_seq, workspace, out_latent, lse, dev_err);
 
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaSuccess;
@@ -182,6 +192,62 @@ mla_status mla_output(const mla_config* cfg, const float* out_latent, const void
     return from_cuda(launch_output_tc(*cfg, out_latent, w_uv, o, n_tokens, dev_err,
                                       (cudaStream_t)stream));
   return from_cuda(launch_output(*cfg, out_latent, w_uv, o, n_tokens, (cudaStream_t)stream));
+}
+
+mla_status mla_decode_step(const mla_config* cfg, const void* q_nope, const void* q_rope,
+                           const void* w_uk, const void* ckv_raw, const void* krope_raw,
+                           const float* gamma, const int32_t* seq_idx, const int32_t* pos,
+                           const int32_t* block_table, int32_t max_blocks, void* pool,
+                           int32_t num_blocks, const int32_t* seq_lens, int32_t batch,
+                           int32_t q_per_seq, void* q_work, void* workspace,
+                           size_t workspace_bytes, float* out_latent, float* lse,
+                           const void* w_uv, void* o, uint32_t* dev_err, void* stream) {
+  // Every argument is checked as the four calls check theirs, before anything is launched.
+  if (!valid_config(cfg) || batch < 0 || q_per_seq < 1) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  const bool rope = cfg->rope_dim > 0;
+  if (!q_nope || (rope && !q_rope) || !w_uk || !ckv_raw || (rope && !krope_raw) || !gamma ||
+      !seq_idx || !pos || !block_table || !pool || !seq_lens || !q_work || !workspace ||
+      !out_latent || !w_uv || !o || !dev_err)
+    return MLA_ERR_INVALID_ARG;
+  if (max_blocks < 1 || num_blocks < 1) return MLA_ERR_INVALID_ARG;
+  const int64_t n64 = (int64_t)batch * q_per_seq;
+  if (n64 > (1 << 24)) return MLA_ERR_UNSUPPORTED;
+  const int n = (int)n64;
+  const size_t need = mla_decode_workspace_size(cfg, batch, q_per_seq);
+  if (need == 0) return MLA_ERR_INVALID_ARG;
+  if (workspace_bytes < need || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+  if (!aligned(pool, 16) || !aligned(q_work, 16) || !aligned(out_latent, 16))
+    return MLA_ERR_INVALID_ARG;
+  const bool simt = cfg->decode_kernel == MLA_DECODE_SIMT;
+  const bool attend_tc = !simt && tc_supported(*cfg);
+  if (cfg->decode_kernel == MLA_DECODE_TENSOR && !tc_supported(*cfg)) return MLA_ERR_UNSUPPORTED;
+  // the fused launches: tensor-core absorb, attention and output, 16-byte aligned operands
+  const bool fused = attend_tc && absorb_tc_supported(*cfg) && output_tc_supported(*cfg) &&
+                     aligned(q_nope, 16) && aligned(w_uk, 16) && aligned(q_rope, 16) &&
+                     aligned(w_uv, 16);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!fused) {
+    // the four calls' own kernels, in order (each validates as above and cannot fail here)
+    mla_status s = mla_absorb_query(cfg, q_nope, q_rope, pos, w_uk, q_work, n, dev_err, stream);
+    if (s == MLA_OK)
+      s = mla_append_latent(cfg, ckv_raw, krope_raw, gamma, seq_idx, pos, block_table, batch,
+                            max_blocks, pool, num_blocks, n, dev_err, stream);
+    if (s == MLA_OK)
+      s = mla_decode(cfg, q_work, pool, block_table, max_blocks, num_blocks, seq_lens, batch,
+                     q_per_seq, workspace, workspace_bytes, out_latent, lse, dev_err, stream);
+    if (s == MLA_OK) s = mla_output(cfg, out_latent, w_uv, o, n, dev_err, stream);
+    return s;
+  }
+  const DecodeParams p = make_params(cfg, q_work, pool, block_table, max_blocks, num_blocks,
+                                     seq_lens, batch, q_per_seq, workspace, out_latent, lse,
+                                     dev_err);
+  cudaError_t e = launch_step_prep(*cfg, q_nope, q_rope, pos, w_uk, q_work, n, ckv_raw,
+                                   krope_raw, gamma, seq_idx, p, pool, st);
+  if (e == cudaSuccess) e = launch_attend_tc(*cfg, p, st);
+  if (e == cudaSuccess) e = launch_combine(p, st);
+  if (e == cudaSuccess) e = launch_output_tc(*cfg, out_latent, w_uv, o, n, dev_err, st);
+  return from_cuda(e);
 }
 
 }  // extern "C"

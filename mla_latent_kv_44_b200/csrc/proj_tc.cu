@@ -16,7 +16,9 @@
 // bounded) for the copies and MMAs already issued, frees TMEM and returns without storing.
 #include <algorithm>
 
+#include "append_row.cuh"
 #include "common.cuh"
+#include "plan_body.cuh"
 #include "tc_ptx.cuh"
 #include "tma_map.h"
 
@@ -84,13 +86,13 @@ struct AbsorbArgs {
   float base;
 };
 
-__global__ void __launch_bounds__(128)
-absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
-                 const AbsorbArgs a) {
-  extern __shared__ uint8_t smem_raw[];
+// One CTA's work: token tile bx, latent tile jt, head h of a grid of (.., ny, nz) tiles.
+__device__ __forceinline__ void absorb_tile(const CUtensorMap* tm_w, const CUtensorMap* tm_q,
+                                            const AbsorbArgs& a, int bx, int jt, int h, int ny,
+                                            int nz, uint8_t* smem_raw) {
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int jt = blockIdx.y, h = blockIdx.z, n0 = blockIdx.x * a.tile;
+  const int n0 = bx * a.tile;
   const int ntok = min(a.tile, a.n - n0);
   const int nmma = round_up(ntok, 16);
   const int ksl = a.dh / kSlab;                      // K slabs of the query rows
@@ -122,20 +124,20 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
   if (threadIdx.x == 0) {
     mbar_expect_tx(bar_full, halves * slab_a + ksl * (uint32_t)a.tile * 128);
     for (int hf = 0; hf < halves; ++hf)
-      tma_load(sA + hf * slab_a, &tm_w, bar_full, j0 + kSlab * hf, h * a.dh);
+      tma_load(sA + hf * slab_a, tm_w, bar_full, j0 + kSlab * hf, h * a.dh);
     for (int k = 0; k < ksl; ++k)
-      tma_load(sB + k * slab_b, &tm_q, bar_full, h * a.dh + kSlab * k, n0);
+      tma_load(sB + k * slab_b, tm_q, bar_full, h * a.dh + kSlab * k, n0);
   }
 
   // RoPE part of the query, while the copies are in flight: pairs (2i, 2i+1) rotated by
   // pos * base^(-2i/d_r), angle and rotation in double. The angles depend on the token only, so
   // each token of this tile is given to one CTA of the tile (CTA (jt, h) takes the tokens
-  // t = jt + gridDim.y * h, ...), which takes the d_r/2 sin/cos pairs once into shared memory
+  // t = jt + ny * h, ...), which takes the d_r/2 sin/cos pairs once into shared memory
   // and rotates the token's query in every head.
   const int D = a.r + a.dr;
   const int half = a.dr / 2;
   double* cs_tab = (double*)(ctl + 64);  // [2][half] cos, sin
-  for (int t = jt + gridDim.y * h; t < ntok; t += gridDim.y * gridDim.z) {
+  for (int t = jt + ny * h; t < ntok; t += ny * nz) {
     const int n = n0 + t;
     __syncthreads();  // the previous token's table is no longer read
     for (int i = threadIdx.x; i < half; i += blockDim.x)
@@ -218,6 +220,62 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant
   if (warp == 1) tmem_free_cols(tmem);
 }
 
+__global__ void __launch_bounds__(128)
+absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
+                 const AbsorbArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  absorb_tile(&tm_w, &tm_q, a, blockIdx.x, blockIdx.y, blockIdx.z, gridDim.y, gridDim.z, smem_raw);
+}
+
+// ------------------------------------------------------------------------------------------
+// The fused step's first launch. Absorbing the query, appending the new cache rows and
+// planning the decode do not depend on one another, so they run as CTA roles of one grid
+// instead of three launches that wait for each other: CTA 0 runs the planner (the longest
+// serial job, so it starts first), CTAs 1 .. app_ctas append four rows each (one warp per
+// row), and the rest are the absorbed query's tiles. Each role waits for the previous grid
+// on the stream before it touches global memory.
+// ------------------------------------------------------------------------------------------
+constexpr int kPrepThreads = 128;
+
+struct PrepArgs {
+  AbsorbArgs ab;             // absorb (n tokens; pos and base shared with the append)
+  int ax, ay, az;            // the absorb tiles: token tiles x latent tiles x heads
+  const __nv_bfloat16* ckv;  // append: raw rows (n, r) and (n, d_r), gain, sequence of each
+  const __nv_bfloat16* kr;
+  const float* gamma;
+  const int32_t* seq;
+  __nv_bfloat16* pool;
+  int app_ctas;
+  float eps;
+  bool vec;
+  DecodeParams p;            // the planner's, and the cache shape for the append
+};
+
+__global__ void __launch_bounds__(kPrepThreads)
+step_prep_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
+                 const PrepArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_a[32], s_b[32], s_carry[2];
+  int id = (int)blockIdx.x;
+  if (id == 0) {
+    plan_body<kPrepThreads>(a.p, s_a, s_b, s_carry);
+    return;
+  }
+  id -= 1;
+  if (id < a.app_ctas) {
+    const int row = id * (kPrepThreads / 32) + (int)(threadIdx.x >> 5);
+    wait_prior_grid();
+    if (row < a.ab.n)
+      append_row<__nv_bfloat16>(row, threadIdx.x & 31, a.ckv, a.kr, a.gamma, a.seq, a.ab.pos,
+                                a.p.table, a.p.batch, a.p.max_blocks, a.pool, a.p.num_blocks,
+                                a.p.r, a.p.dr, a.p.bs, a.eps, a.ab.base, a.p.err, a.vec);
+    return;
+  }
+  id -= a.app_ctas;
+  const int x = id % a.ax, y = (id / a.ax) % a.ay, z = id / (a.ax * a.ay);
+  absorb_tile(&tm_w, &tm_q, a.ab, x, y, z, a.ay, a.az, smem_raw);
+}
+
 // ------------------------------------------------------------------------------------------
 // Output. Grid (token tiles, ceil(d_v / 128), H); 256 threads. The K = r contraction runs in
 // chunks of 128 latent dims through two shared-memory stages: TMA brings W_UV[h][i0:i0+128,
@@ -254,7 +312,6 @@ output_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const OutputArgs a) {
   uint32_t* tmem_slot = (uint32_t*)(ctl + 32);
   int* flags = (int*)(ctl + 48);          // [0] chunks whose MMAs were committed, [1] loaded
   const int nchunks = (a.r + 127) / 128;
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_full + 8 * s, 1);
@@ -269,11 +326,10 @@ output_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const OutputArgs a) {
   __syncthreads();
   tc_after();
   const uint32_t tmem = *tmem_slot;
-  wait_prior_grid();
-
   // The weights of chunk c go by TMA into stage c & 1 as soon as that stage is free (chunks 0
-  // and 1 at once). The latent of chunk c + 1 is loaded into registers while chunk c's MMAs
-  // run: each thread holds kOutItems groups of 8 floats (tile <= 64 tokens x 16 groups).
+  // and 1 at once, before anything else reads memory). The latent of chunk c + 1 is loaded into
+  // registers while chunk c's MMAs run: each thread holds kOutItems groups of 8 floats
+  // (tile <= 64 tokens x 16 groups).
   auto issue_w = [&](int c) {
     const int s = c & 1;
     const int k0 = c * 128, nsl = min(128, a.r - k0) / kSlab;
@@ -283,6 +339,11 @@ output_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const OutputArgs a) {
                h * a.dv + i0);
     flags[1] = c + 1;
   };
+  wait_prior_grid();
+  if (threadIdx.x == 0) {
+    issue_w(0);
+    if (nchunks > 1) issue_w(1);
+  }
   float4 pf[2 * kOutItems];
   auto load_lat = [&](int c) {
     const int k0 = c * 128, groups = min(128, a.r - k0) / 8;
@@ -299,10 +360,6 @@ output_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const OutputArgs a) {
       }
     }
   };
-  if (threadIdx.x == 0) {
-    issue_w(0);
-    if (nchunks > 1) issue_w(1);
-  }
   load_lat(0);
 
   bool ok = true;
@@ -475,6 +532,44 @@ cudaError_t launch_output_tc(const mla_config& c, const float* lat, const void* 
   OutputArgs a{lat, (__nv_bfloat16*)o, err, n, H, dv, r, tile};
   dim3 grid((n + tile - 1) / tile, mts, H);
   return launch_pdl(output_tc_kernel, grid, dim3(256), smem, st, tw, a);
+}
+
+cudaError_t launch_step_prep(const mla_config& c, const void* q_nope, const void* q_rope,
+                             const int32_t* pos, const void* w_uk, void* q_out, int n,
+                             const void* ckv, const void* kr, const float* gamma,
+                             const int32_t* seq, const DecodeParams& p, void* pool,
+                             cudaStream_t st) {
+  const int H = c.num_heads, dh = c.head_dim, r = c.kv_rank;
+  const int jts = (r + kWRows - 1) / kWRows;
+  const int tile = token_tile(n, jts * H, kMaxTokTile);
+  CUtensorMap tw, tq;
+  if (!make_bf16_map(&tw, w_uk, (uint64_t)r, (uint64_t)H * dh, (uint64_t)r * 2, (uint32_t)dh) ||
+      !make_bf16_map(&tq, q_nope, (uint64_t)H * dh, (uint64_t)n, (uint64_t)H * dh * 2,
+                     (uint32_t)tile))
+    return cudaErrorInvalidValue;
+  const size_t smem = absorb_smem(dh, c.rope_dim, tile);
+  cudaError_t e = cudaFuncSetAttribute(step_prep_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  PrepArgs a;
+  a.ab = AbsorbArgs{(const __nv_bfloat16*)q_rope, pos, (__nv_bfloat16*)q_out, p.err, n, H, dh, r,
+                    c.rope_dim, tile, c.rope_base};
+  a.ax = (n + tile - 1) / tile;
+  a.ay = jts;
+  a.az = H;
+  a.ckv = (const __nv_bfloat16*)ckv;
+  a.kr = (const __nv_bfloat16*)kr;
+  a.gamma = gamma;
+  a.seq = seq;
+  a.pool = (__nv_bfloat16*)pool;
+  a.app_ctas = (n + kPrepThreads / 32 - 1) / (kPrepThreads / 32);
+  a.eps = c.rms_eps;
+  a.vec = c.kv_rank % 256 == 0 && c.kv_rank <= 1024 && ((uintptr_t)ckv & 15) == 0 &&
+          ((uintptr_t)gamma & 15) == 0 && ((uintptr_t)pool & 15) == 0 &&
+          ((c.kv_rank + c.rope_dim) * 2) % 16 == 0;
+  a.p = p;
+  const int grid = 1 + a.app_ctas + a.ax * a.ay * a.az;
+  return launch_pdl(step_prep_kernel, dim3(grid), dim3(kPrepThreads), smem, st, tw, tq, a);
 }
 
 }  // namespace mla

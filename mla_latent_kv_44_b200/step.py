@@ -15,7 +15,7 @@ import torch
 import mla_inputs as mi
 
 from . import (DECODE_AUTO, STAGES_ALL, Config, absorb_query, append_latent, decode,
-               decode_workspace_size, output)
+               decode_step, decode_workspace_size, output)
 
 POOL_SENTINEL = -1  # every bit set: NaN in both bf16 and fp32
 
@@ -145,10 +145,27 @@ class DecodeState:
         output(self.cfg, self.out_latent, self.w_uv, self.o, stream, self.dev_err)
 
     def step(self, stream=None):
+        """The four calls of the hot path, one after another."""
         self.absorb(stream)
         self.append(stream)
         self.attend(stream)
         self.project(stream)
+
+    def fused_launches(self) -> int:
+        """Kernel launches of step_fused: 4 where mla_decode_step fuses (bf16, the tensor-core
+        attention shape, tensor-core projections), else the four calls' 6."""
+        c = self.cfg
+        fused = (c.dtype == "bf16" and c.decode_kernel != 1 and c.num_heads == 128 and
+                 c.kv_rank == 512 and c.rope_dim == 64 and c.block_size == 64 and
+                 c.head_dim % 64 == 0 and c.head_dim <= 256)
+        return 4 if fused else 6
+
+    def step_fused(self, stream=None):
+        """The same step through mla_decode_step (one call; four launches where it can)."""
+        decode_step(self.cfg, self.q_nope, self.q_rope, self.w_uk, self.ckv_new, self.krope_new,
+                    self.gamma, self.seq_new, self.pos_new, self.block_table, self.pool,
+                    self.seq_lens, self.w.new_tokens, self.q, self.workspace, self.out_latent,
+                    self.lse, self.w_uv, self.o, self.dev_err, stream)
 
     # ---- helpers ------------------------------------------------------------------------
     def sequence_rows(self, b: int) -> np.ndarray:
