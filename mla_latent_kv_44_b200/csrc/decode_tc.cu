@@ -81,7 +81,7 @@ constexpr int kPSlots = 4;
 constexpr int kSlotBytes = kPBlockBytes + kHdrBytes;          // 17 KB (1 KB aligned)
 constexpr int kV_V = 0;
 constexpr int kV_P = kV_V + kVStages * kVStageBytes;          // 128 KB
-// output staging: per epilogue warp one 4 KB box of 32 rows x 32 fp32 (a TMA store source)
+// output staging: per epilogue warp one 4 KB box of 32 rows x 32 fp32 (a transpose buffer)
 constexpr int kOutBoxBytes = 32 * 32 * 4;
 constexpr int kV_Out = kV_P + kPSlots * kSlotBytes;           // 196 KB (1 KB aligned)
 constexpr int kV_End = kV_Out + 4 * kOutBoxBytes;             // 212 KB
@@ -253,9 +253,7 @@ struct BlockWindow {
 
 __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(168)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
-                 const __grid_constant__ CUtensorMap tm_q,
-                 const __grid_constant__ CUtensorMap tm_out,
-                 const __grid_constant__ CUtensorMap tm_part, const DecodeParams p) {
+                 const __grid_constant__ CUtensorMap tm_q, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t s_base = saddr(smem);
@@ -797,46 +795,56 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
         if (!wait_pv(t)) break;
         tc_after();
         const float inv_l = 1.f / l;
-        // O / l leaves through shared memory: each warp stages its 32 rows x 32 columns as a
-        // 128-byte-swizzled 4 KB box and one lane stores the box with TMA, so the global
-        // writes are whole lines rather than 16-byte pieces 2 KB apart.
-        // kept in L2: the combine (partials) and the output projection (O) read them next,
-        // after the rest of the cache has streamed through
+        // O / l leaves through shared memory: each warp stages its 32 rows x 32 columns in a
+        // 4 KB box (row = lane, 16-byte groups swizzled by row % 8), reads it back four rows
+        // per instruction and stores whole 128-byte lines; the box is free again as soon as
+        // the warp has read it, so no store is waited for. Kept in L2: the combine (partials)
+        // and the output projection (O) read them next, after the rest of the cache has
+        // streamed through.
         const uint64_t keep = l2_evict_last();
-        const CUtensorMap* map = tl.slot < 0 ? &tm_out : &tm_part;
-        const int row0 = (tl.slot < 0 ? tl.bt : tl.slot) * kH + quad * 32;
+        float* dst = (tl.slot < 0 ? p.out + (size_t)tl.bt * kH * kR
+                                  : p.part_o + (size_t)tl.slot * kH * kR) +
+                     (size_t)(quad * 32 + (lane >> 3)) * kR + 4 * (lane & 7);
         const uint32_t box = s_base + kV_Out + (uint32_t)quad * kOutBoxBytes;
+        const uint32_t wrow = box + (uint32_t)lane * 128;
+        // read-back: instruction i takes rows 4i .. 4i + 3, lane: row 4i + lane / 8, 16-byte
+        // group lane % 8, stored at group (lane % 8) ^ (row % 8) with row % 8 = lane / 8 for
+        // even i and lane / 8 + 4 for odd i
+        const uint32_t g = (uint32_t)((lane & 7) ^ (lane >> 3));
+        const uint32_t rd_even = box + (uint32_t)(lane >> 3) * 128 + 16u * g;
+        const uint32_t rd_odd = box + (uint32_t)(lane >> 3) * 128 + 16u * (g ^ 4u);
         // the next chunk's TMEM load is in flight while this chunk is staged and stored
         uint32_t o[32], nx[32];
         tmem_ld32(tq, o);
 #pragma unroll 1
         for (int ch = 0; ch < 16; ++ch) {
           if (ch + 1 < 16) tmem_ld32_async(tq + 32 * (ch + 1), nx);
-          if (ch >= 1) {  // the previous chunk's store is done reading the box
-            if (lane == 0) bulk_wait_read<0>();
-            __syncwarp();
-          }
-          const uint32_t row = box + (uint32_t)lane * 128;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             row + 16u * (uint32_t)(u ^ (lane & 7))),
+                             wrow + 16u * (uint32_t)(u ^ (lane & 7))),
                          "f"(__uint_as_float(o[4 * u]) * inv_l),
                          "f"(__uint_as_float(o[4 * u + 1]) * inv_l),
                          "f"(__uint_as_float(o[4 * u + 2]) * inv_l),
                          "f"(__uint_as_float(o[4 * u + 3]) * inv_l)
                          : "memory");
-          fence_proxy_async();
           __syncwarp();
-          if (lane == 0) tma_store_hint(map, box, 32 * ch, row0, keep);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 x;
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
+                         : "r"(((i & 1) ? rd_odd : rd_even) + 512u * (uint32_t)i)
+                         : "memory");
+            st_global_hint(dst + (size_t)(4 * i) * kR + 32 * ch, x, keep);
+          }
+          __syncwarp();  // the box is read before the next chunk overwrites it
           if (ch + 1 < 16) {
             tmem_wait_ld(nx);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = nx[i];
           }
         }
-        if (lane == 0) bulk_wait_read<0>();  // the box is free for the next segment
-        __syncwarp();
         tc_before();
       }
       g += tl.nb;
@@ -845,7 +853,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
   }
 
   // ---------------------------------------------------------------------- teardown
-  if (!score && warp >= 2 && warp < 6 && lane == 0) bulk_wait_all();  // output stores landed
   // The score CTA tells the value CTA how many P blocks it sent, so that the value CTA can
   // wait (bounded) for any that are still landing in its shared memory before either exits.
   if (score && warp == 10 && lane == 0)
@@ -887,11 +894,9 @@ bool tc_supported(const mla_config& c) {
 
 cudaError_t launch_attend_tc(const mla_config& c, const DecodeParams& p, cudaStream_t st) {
   (void)c;
-  CUtensorMap kv, qm, om, pm;
+  CUtensorMap kv, qm;
   if (!make_bf16_map(&kv, p.pool, kD, (uint64_t)p.num_blocks * kRows, kD * 2, kRows) ||
-      !make_bf16_map(&qm, p.q, kD, (uint64_t)p.BT * kH, kD * 2, kH) ||
-      !make_f32_box32_map(&om, p.out, kR, (uint64_t)p.BT * kH) ||
-      !make_f32_box32_map(&pm, p.part_o, kR, (uint64_t)kMaxPartials * kH))
+      !make_bf16_map(&qm, p.q, kD, (uint64_t)p.BT * kH, kD * 2, kH))
     return cudaErrorInvalidValue;
   // the shared-memory attribute applies to the device current when it is set: once per device
   static std::atomic<unsigned long long> attr_devices{0};
@@ -906,7 +911,7 @@ cudaError_t launch_attend_tc(const mla_config& c, const DecodeParams& p, cudaStr
     attr_devices.fetch_or(bit, std::memory_order_acq_rel);
   }
   return launch_pdl(attend_tc_kernel, dim3(2 * kRanges), dim3(kThreads), kSmemBytes, st, kv, qm,
-                    om, pm, p);
+                    p);
 }
 
 }  // namespace mla

@@ -73,21 +73,6 @@ __device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst), "l"(map), "r"(bar), "r"(x), "r"(y)
       : "memory");
 }
-// shared::cta -> global tiled TMA store of one box, tracked in this thread's bulk group
-__device__ __forceinline__ void tma_store(const CUtensorMap* map, uint32_t src, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];\n\t"
-      "cp.async.bulk.commit_group;" ::"l"(map), "r"(src), "r"(x), "r"(y)
-      : "memory");
-}
-// tma_store with an L2 cache policy (createpolicy) for the written lines
-__device__ __forceinline__ void tma_store_hint(const CUtensorMap* map, uint32_t src, int x, int y,
-                                               uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;\n\t"
-      "cp.async.bulk.commit_group;" ::"l"(map), "r"(src), "r"(x), "r"(y), "l"(policy)
-      : "memory");
-}
 // L2 policy that lets lines go before others (fraction 1.0)
 __device__ __forceinline__ uint64_t l2_evict_first() {
   uint64_t pol;
@@ -109,14 +94,11 @@ __device__ __forceinline__ uint64_t l2_evict_last() {
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
-// wait until at most N of this thread's bulk groups still read shared memory
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-// wait until all of this thread's bulk groups completed (writes visible)
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+// 16-byte global store with an L2 cache policy
+__device__ __forceinline__ void st_global_hint(float* ptr, float4 v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w), "l"(policy)
+               : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -39,18 +39,4 @@ inline bool make_bf16_map(CUtensorMap* m, const void* base, uint64_t cols, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D fp32 view: `rows` rows of `cols` elements (contiguous), moved in 128-byte swizzled boxes
-// of 32 columns x 32 rows (the layout TMA stores read from shared memory).
-inline bool make_f32_box32_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
-  auto fn = tensor_map_encoder();
-  if (!fn || ((uintptr_t)base & 15) || ((cols * 4) & 15)) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
-  cuuint32_t box[2] = {32, 32};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace mla
