@@ -65,12 +65,18 @@ def aggregate_rate(units_per_rank_step: float, world: int, steps: int, elapsed_m
     return units_per_rank_step * world * steps / (elapsed_ms * 1e-3)
 
 
-# DRAM bytes (read + write) of one attention launch on the bench workload, from an ncu capture
-# of that kernel source, keyed by a hash of the kernel's code:
-# when the kernel changes, the figure no longer applies and the bench reports null until it is
-# re-measured.
+# DRAM bytes (read + write) of one attention launch, from an ncu capture of that kernel source
+# on that workload, keyed by the workload and a hash of the kernel's code: when the kernel
+# changes (or another workload runs), the figure does not apply and the bench reports null.
 ATTEND_SOURCES = ("decode_tc.cu", "tc_ptx.cuh", "tma_map.h", "common.cuh")
-ATTEND_TRAFFIC = {"483f7328a205a490": 646_193_152 + 8_178_176}
+ATTEND_TRAFFIC = {("dsv2", "6dea7720cb356fe8"): 644_382_976 + 8_976_896}
+
+
+def attend_traffic(args):
+    """The captured DRAM bytes of the tensor-core attention launch for this run, or None."""
+    if args.decode_kernel == "simt":
+        return None
+    return ATTEND_TRAFFIC.get((args.workload, attend_source_hash()))
 
 
 def attend_source_hash() -> str:
@@ -559,7 +565,7 @@ def run_ours(args, w):
 
     rows = mi.total_rows(w, 0)
     roof, attend_bytes, gbs, tflops = attention_roofline(w, rows, attend_ms, load_peaks(),
-                                                         ATTEND_TRAFFIC.get(attend_source_hash()))
+                                                         attend_traffic(args))
     # per-stage rates of the projections and the append (algorithmic bytes and FLOPs over the
     # per-kernel times of the breakdown run)
     N, H = tokens_per_step, w.num_heads

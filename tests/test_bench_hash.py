@@ -41,3 +41,16 @@ def test_a_code_change_changes_the_key(tmp_path, monkeypatch):
     assert "constexpr int kKStages = 4;" in text
     f.write_text(text.replace("constexpr int kKStages = 4;", "constexpr int kKStages = 3;"))
     assert _hash_at(tmp_path, monkeypatch) != before
+
+
+def test_traffic_applies_to_its_workload_and_kernel_only():
+    import argparse
+
+    (workload, key), traffic = next(iter(bench.ATTEND_TRAFFIC.items()))
+    assert isinstance(traffic, int) and traffic > 0
+    here = bench.attend_source_hash()
+    args = argparse.Namespace(decode_kernel="auto", workload=workload)
+    assert bench.attend_traffic(args) == (traffic if key == here else None)
+    other = [w for w in ("dsv2", "ragged", "mtp") if w != workload][0]
+    assert bench.attend_traffic(argparse.Namespace(decode_kernel="auto", workload=other)) is None
+    assert bench.attend_traffic(argparse.Namespace(decode_kernel="simt", workload=workload)) is None
