@@ -41,6 +41,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-kernel", default="auto", choices=["auto", "simt", "tensor"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--context-parallel", type=int, default=0, metavar="G",
+                    help="time the context-parallel split of a long-context batch into G "
+                         "slices (emulated one after another on this process's GPU)")
     return ap.parse_args()
 
 
@@ -611,10 +614,106 @@ def run_ours(args, w):
     return 0
 
 
+# ---------------------------------------------------------------------------------------
+# Context-parallel split (each sequence's rows cut into G block-aligned slices, one per GPU of
+# a group; every slice decoded by mla_decode, the partials all-gathered and merged by
+# mla_combine_partials). With one GPU the G ranks run one after another on it: each slice's
+# decode and the merge are timed with CUDA events; the exchange between GPUs is not.
+# ---------------------------------------------------------------------------------------
+def run_context_parallel(args):
+    import numpy as np
+    import torch
+
+    import mla_inputs as mi
+    import mla_latent_kv_44_b200 as mla
+    from mla_latent_kv_44_b200 import context_parallel as cp
+    from mla_latent_kv_44_b200.step import DecodeState
+
+    rank, world, local = dist_env()
+    if world > 1:
+        if rank == 0:
+            print(json.dumps({"metric": "context-parallel decode", "unavailable":
+                              "the G ranks are emulated on one GPU; run without torchrun"}))
+        return 0
+    G = args.context_parallel
+    w = mi.scaled(mi.WORKLOADS["dsv2"], batch=8, cached=32767)
+    dev = torch.device("cuda", 0)
+    st = DecodeState(w, device=str(dev), sequences=[])
+    stream = torch.cuda.Stream(device=dev)
+    B, T, H, r = w.batch, w.new_tokens, w.num_heads, w.kv_rank
+    n = B * T
+    with torch.cuda.stream(stream):
+        st.absorb(stream)
+        st.append(stream)
+    plans = [cp.rank_plan(st.layout.table, st.rows, T, G, k, st.layout.block_size)
+             for k in range(G)]
+    tables = [torch.from_numpy(p.table).to(dev) for p in plans]
+    lens = [torch.from_numpy(p.lens).to(dev) for p in plans]
+    wss = [torch.empty(mla.decode_workspace_size(st.cfg, len(p.lens), p.q_per_seq),
+                       dtype=torch.uint8, device=dev) for p in plans]
+    parts_o = torch.empty((G, n, H, r), device=dev)
+    parts_l = torch.empty((G, n, H), device=dev)
+
+    def one_step(ev=None):
+        for k, p in enumerate(plans):
+            if ev is not None:
+                ev[k][0].record(stream)
+            mla.decode(st.cfg, st.q, st.pool, tables[k], lens[k], p.q_per_seq, wss[k],
+                       parts_o[k], parts_l[k], st.dev_err, stream)
+            if ev is not None:
+                ev[k][1].record(stream)
+        if ev is not None:
+            ev[G][0].record(stream)
+        mla.combine_partials(st.cfg, parts_o, parts_l, st.out_latent, st.lse, stream)
+        if ev is not None:
+            ev[G][1].record(stream)
+
+    props = torch.cuda.get_device_properties(dev)
+    clock = ClockSampler(str(getattr(props, "uuid", "")), 0)
+    clock.start()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            one_step()
+    stream.synchronize()
+    evs = []
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(G + 1)]
+            one_step(ev)
+            evs.append(ev)
+    stream.synchronize()
+    clock.stop()
+    if int(st.dev_err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(st.dev_err.item())}")
+    per = np.array([[e[k][0].elapsed_time(e[k][1]) * 1e3 for k in range(G + 1)] for e in evs])
+    slice_us = per[:, :G].mean(axis=0)
+    merge_us = float(per[:, G].mean())
+    step_us = float(slice_us.max()) + merge_us
+    rows_total = int(np.sum(st.rows))
+    print(json.dumps({
+        "metric": "context-parallel decode tokens/s (slowest slice + merge; exchange excluded)",
+        "value": n / (step_us * 1e-6), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"dsv2-long: H=128 r=512 d_r=64 B={B} S={int(st.rows[0])} T={T} "
+                               f"bf16 paged 64-row blocks", "slices": G,
+                   "emulated": "G slices one after another on one GPU"},
+        "slice_us": [round(float(x), 2) for x in slice_us],
+        "slice_rows": [int(np.sum(p.lens) // (1 if p.q_per_seq == T else T)) for p in plans],
+        "merge_us": merge_us,
+        "exchange_bytes_per_rank": n * H * (r + 1) * 4,
+        "single_gpu_rows_per_step": rows_total,
+        "clocks": clock.summary(t0, time.time(), "warm-up and timed steps"),
+    }), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     import mla_inputs as mi
 
+    if args.context_parallel:
+        return run_context_parallel(args)
     w = mi.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)

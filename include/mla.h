@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 3
+#define MLA_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define MLA_API __attribute__((visibility("default")))
@@ -236,6 +236,34 @@ MLA_API mla_status mla_decode_step(const mla_config* cfg, const void* q_nope, co
                                    int32_t q_per_seq, void* q_work, void* workspace,
                                    size_t workspace_bytes, float* out_latent, float* lse,
                                    const void* w_uv, void* o, uint32_t* dev_err, void* stream);
+
+/* Most parts mla_combine_partials merges in one call. */
+#define MLA_MAX_COMBINE_PARTS 256
+
+/*
+ * mla_combine_partials -- merge partial decode results of the same row groups computed over
+ * disjoint sets of each sequence's cache rows: the per-GPU results of a context-parallel
+ * split, where every GPU holds a contiguous slice of each sequence's rows, runs mla_decode on
+ * its slice, and the slices' (out_latent, lse) are gathered. The merge is the one mla_decode
+ * applies to its own work ranges: a softmax over all rows equals the softmaxes over disjoint
+ * row sets weighted by their shares of the normaliser ([B] Absorbing projections: attend
+ * directly to latents; "MLA from scratch in PyTorch", Memory comparison: the cache of long
+ * contexts outgrows one GPU). For row group k < n and head h:
+ *   L = log(sum_i exp(part_lse[i, k, h])),
+ *   out_latent[k, h, :] = sum_i exp(part_lse[i, k, h] - L) * part_latent[i, k, h, :],
+ *   lse[k, h] = L.
+ * part_latent (parts, n, H, r) float32 and part_lse (parts, n, H) float32, part-major, each
+ * part as mla_decode writes out_latent and lse; out_latent (n, H, r) float32; lse (n, H)
+ * float32 or NULL. part_latent and out_latent must be 16-byte aligned; out_latent must not
+ * overlap the parts. 1 <= parts <= MLA_MAX_COMBINE_PARTS. A part whose lse is -inf holds no
+ * rows and is skipped (its part_latent is not read); a row group with no rows in any part gets
+ * 0 and lse -inf. fp32 arithmetic in part order: the same inputs give the same bits.
+ * MLA_ERR_INVALID_ARG for a bad config, a null pointer, misalignment or parts out of range;
+ * n == 0 returns MLA_OK without launching.
+ */
+MLA_API mla_status mla_combine_partials(const mla_config* cfg, const float* part_latent,
+                                        const float* part_lse, int32_t parts, int32_t n,
+                                        float* out_latent, float* lse, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 MLA_API const char* mla_status_string(mla_status status);

@@ -25,6 +25,7 @@ DECODE_AUTO, DECODE_SIMT, DECODE_TENSOR = 0, 1, 2
 DEV_OOB_BLOCK, DEV_OOB_POS, DEV_WAIT_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
 STAGE_PLAN, STAGE_ATTEND, STAGE_COMBINE = 1, 2, 4
 STAGES_ALL = STAGE_PLAN | STAGE_ATTEND | STAGE_COMBINE
+MAX_COMBINE_PARTS = 256  # MLA_MAX_COMBINE_PARTS
 
 _c_i32, _c_f32, _vp, _sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -63,6 +64,7 @@ def _load():
         "mla_decode_step": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _vp,
                                      _c_i32, _vp, _c_i32, _c_i32, _vp, _vp, _sz, _vp, _vp, _vp,
                                      _vp, _vp, _vp]),
+        "mla_combine_partials": (_c_i32, [P, _vp, _vp, _c_i32, _c_i32, _vp, _vp, _vp]),
         "mla_status_string": (ctypes.c_char_p, [_c_i32]),
         "mla_abi_version": (_c_i32, []),
     }
@@ -213,6 +215,16 @@ def output(cfg: Config, out_latent, w_uv, o, stream=None, dev_err=None):
     c = cfg.c()
     _check(lib.mla_output(ctypes.byref(c), _ptr(out_latent), _ptr(w_uv), _ptr(o),
                           int(out_latent.shape[0]), _ptr(dev_err), _stream(stream)), "mla_output")
+
+
+def combine_partials(cfg: Config, part_latent, part_lse, out_latent, lse=None, stream=None):
+    """mla_combine_partials: merge part_latent (parts, n, H, r) / part_lse (parts, n, H), each
+    part a decode over a disjoint set of the rows, into out_latent (n, H, r) and lse (n, H)."""
+    c = cfg.c()
+    _check(lib.mla_combine_partials(ctypes.byref(c), _ptr(part_latent), _ptr(part_lse),
+                                    int(part_latent.shape[0]), int(part_latent.shape[1]),
+                                    _ptr(out_latent), _ptr(lse), _stream(stream)),
+           "mla_combine_partials")
 
 
 def abi_version() -> int:

@@ -83,4 +83,72 @@ cudaError_t launch_combine(const DecodeParams& p, cudaStream_t st) {
   return launch_pdl(combine_kernel, grid, dim3(128), 0, st, p);
 }
 
+// ------------------------------------------------------------------------------------------
+// Merge of results computed apart: `parts` softmax-normalised partial results of the same n
+// row groups over disjoint sets of cache rows (one per GPU of a context-parallel split of
+// every sequence's rows), laid out part-major: o (parts, n, H, r), lse (parts, n, H). The
+// same log-sum-exp merge as above, in part order. A part with lse = -inf holds no rows and is
+// skipped whatever its o; a row group with no rows in any part gets 0 and -inf.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kCombineHeads * 32)
+combine_parts_kernel(const float* part_o, const float* part_lse, int parts, int n, int H, int r,
+                     float* out, float* lse) {
+  __shared__ float s_w[kCombineHeads][MLA_MAX_COMBINE_PARTS];
+  wait_prior_grid();
+  const int bt = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * kCombineHeads + warp;
+  if (h >= H) return;
+  const size_t plane = (size_t)n * H;  // one part's (n, H) entries
+  const size_t at = (size_t)bt * H + h;
+  float mx = -INFINITY;
+  for (int k = lane; k < parts; k += 32) mx = fmaxf(mx, part_lse[k * plane + at]);
+  mx = warp_max(mx);
+  float4* dst = (float4*)(out + at * r);
+  const int r4 = r / 4;
+  if (mx == -INFINITY) {
+    for (int d = lane; d < r4; d += 32) dst[d] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane == 0 && lse) lse[at] = -INFINITY;
+    return;
+  }
+  float z = 0.f;
+  for (int k = lane; k < parts; k += 32) z += expf(part_lse[k * plane + at] - mx);
+  z = warp_sum(z);
+  const float L = mx + logf(z);
+  for (int k = lane; k < parts; k += 32) s_w[warp][k] = expf(part_lse[k * plane + at] - L);
+  __syncwarp();
+  for (int d0 = lane; d0 < r4; d0 += 128) {
+    float4 acc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < parts; ++k) {
+      const float w = s_w[warp][k];
+      if (w == 0.f) continue;  // an empty part (or one far below the others)
+      const float4* src = (const float4*)(part_o + (k * plane + at) * r);
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        v[u] = (d0 + 32 * u < r4) ? __ldcs(src + d0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc[u].x = fmaf(w, v[u].x, acc[u].x);
+        acc[u].y = fmaf(w, v[u].y, acc[u].y);
+        acc[u].z = fmaf(w, v[u].z, acc[u].z);
+        acc[u].w = fmaf(w, v[u].w, acc[u].w);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (d0 + 32 * u < r4) dst[d0 + 32 * u] = acc[u];
+  }
+  if (lane == 0 && lse) lse[at] = L;
+}
+
+cudaError_t launch_combine_parts(const float* part_o, const float* part_lse, int parts, int n,
+                                 int H, int r, float* out, float* lse, cudaStream_t st) {
+  dim3 grid(n, (H + kCombineHeads - 1) / kCombineHeads);
+  return launch_pdl(combine_parts_kernel, grid, dim3(kCombineHeads * 32), 0, st, part_o,
+                    part_lse, parts, n, H, r, out, lse);
+}
+
 }  // namespace mla

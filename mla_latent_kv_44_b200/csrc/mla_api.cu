@@ -7,6 +7,12 @@
 
 using namespace mla;
 
+namespace mla {
+// decode_plan.cu: the merge behind mla_combine_partials
+cudaError_t launch_combine_parts(const float* part_o, const float* part_lse, int parts, int n,
+                                 int H, int r, float* out, float* lse, cudaStream_t st);
+}  // namespace mla
+
 namespace {
 
 bool valid_config(const mla_config* c) {
@@ -84,6 +90,18 @@ const char* mla_status_string(mla_status s) {
 }
 
 int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
+
+mla_status mla_combine_partials(const mla_config* cfg, const float* part_latent,
+                                const float* part_lse, int32_t parts, int32_t n,
+                                float* out_latent, float* lse, void* stream) {
+  if (!valid_config(cfg) || parts < 1 || parts > MLA_MAX_COMBINE_PARTS || n < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (n == 0) return MLA_OK;
+  if (!part_latent || !part_lse || !out_latent) return MLA_ERR_INVALID_ARG;
+  if (!aligned(part_latent, 16) || !aligned(out_latent, 16)) return MLA_ERR_INVALID_ARG;
+  return from_cuda(launch_combine_parts(part_latent, part_lse, parts, n, cfg->num_heads,
+                                        cfg->kv_rank, out_latent, lse, (cudaStream_t)stream));
+}
 
 mla_status mla_absorb_query(const mla_config* cfg, const void* q_nope, const void* q_rope,
                             const int32_t* pos, const void* w_uk, void* q_out, int32_t n_tokens,

@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(mla):
 
 
 def test_abi_version_and_status_strings(mla):
-    assert mla.abi_version() == 3
+    assert mla.abi_version() == 4
     assert mla.status_string(0) == "MLA_OK"
     assert mla.status_string(4) == "MLA_ERR_WORKSPACE"
     assert mla.status_string(99) == "MLA_ERR_UNKNOWN"
@@ -150,3 +150,21 @@ def test_static_workspace_entry_point_returns_mla_decodes_statuses(mla):
     st = mla.lib.mla_decode_static_workspace(ctypes.byref(good), 256, 256, 256, 4, 4, 256, big, 1,
                                              256, None, 256, None)
     assert st == mla.MLA_ERR_WORKSPACE
+
+
+def test_combine_partials_validates_arguments(mla):
+    c = _cfg(mla)
+    f = mla.lib.mla_combine_partials
+    assert f(ctypes.byref(c), 256, 256, 0, 4, 256, None, None) == mla.MLA_ERR_INVALID_ARG
+    assert f(ctypes.byref(c), 256, 256, mla.MAX_COMBINE_PARTS + 1, 4, 256, None,
+             None) == mla.MLA_ERR_INVALID_ARG
+    assert f(ctypes.byref(c), None, 256, 2, 4, 256, None, None) == mla.MLA_ERR_INVALID_ARG
+    assert f(ctypes.byref(c), 256, None, 2, 4, 256, None, None) == mla.MLA_ERR_INVALID_ARG
+    assert f(ctypes.byref(c), 256, 256, 2, 4, None, None, None) == mla.MLA_ERR_INVALID_ARG
+    assert f(ctypes.byref(c), 264, 256, 2, 4, 256, None, None) == mla.MLA_ERR_INVALID_ARG
+    assert f(ctypes.byref(c), 256, 256, 2, 4, 260, None, None) == mla.MLA_ERR_INVALID_ARG
+    assert f(ctypes.byref(c), 256, 256, 2, -1, 256, None, None) == mla.MLA_ERR_INVALID_ARG
+    bad = _cfg(mla, kv_rank=48)
+    assert f(ctypes.byref(bad), 256, 256, 2, 4, 256, None, None) == mla.MLA_ERR_INVALID_ARG
+    # no row groups: nothing to do, whatever the pointers
+    assert f(ctypes.byref(c), None, None, 2, 0, None, None, None) == mla.MLA_OK
