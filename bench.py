@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-kernel", default="auto", choices=["auto", "simt", "tensor"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--front", action="store_true",
+                    help="time the decode front end (mla_project) at the workload's shape")
     ap.add_argument("--context-parallel", type=int, default=0, metavar="G",
                     help="time the context-parallel split of a long-context batch into G "
                          "slices (emulated one after another on this process's GPU)")
@@ -708,10 +710,99 @@ def run_context_parallel(args):
     return 0
 
 
+# ---------------------------------------------------------------------------------------
+# Decode front end (mla_project): the projections of one step's hidden states, which stream
+# every front-end weight once (W_DQ, W_QR, W_DKV, W_KR from x; W_UQ from c_q).
+# ---------------------------------------------------------------------------------------
+def run_front(args, w):
+    import numpy as np
+    import torch
+
+    import mla_inputs as mi
+    import mla_latent_kv_44_b200 as mla
+
+    rank, world, local = dist_env()
+    if world > 1:
+        if rank == 0:
+            print(json.dumps({"metric": "decode front end", "unavailable":
+                              "measured on one GPU; run without torchrun"}))
+        return 0
+    dev = torch.device("cuda", 0)
+    n = w.batch * w.new_tokens
+    d = mi.layer_draw(w, 0, x_rows=n)
+    cfg = mla.Config(num_heads=w.num_heads, head_dim=w.head_dim, kv_rank=w.kv_rank,
+                     rope_dim=w.rope_dim, block_size=64, dtype=w.dtype)
+    tdt = cfg.torch_dtype
+
+    def up(a):
+        return None if a is None else torch.from_numpy(
+            np.ascontiguousarray(mi.storage_round(w, a), dtype=np.float32)).to(dev, tdt)
+
+    wq = d.w_dq if w.q_rank else d.w_q
+    x, w_dq, w_uq, w_qr, w_dkv, w_kr = map(up, (d.x, wq, d.w_uq, d.w_qr, d.w_dkv, d.w_kr))
+    gq = None if d.gamma_q is None else torch.from_numpy(d.gamma_q.astype(np.float32)).to(dev)
+    H, dh, dr, r = w.num_heads, w.head_dim, w.rope_dim, w.kv_rank
+    q_nope = torch.empty((n, H, dh), dtype=tdt, device=dev)
+    q_rope = torch.empty((n, H, dr), dtype=tdt, device=dev)
+    ckv = torch.empty((n, r), dtype=tdt, device=dev)
+    kr = torch.empty((n, dr), dtype=tdt, device=dev)
+    front = mla.front_config(w.d_model, w.q_rank or 0, w.rms_eps)
+    ws = torch.empty(mla.project_workspace_size(cfg, front, n), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        mla.project(cfg, front, x, w_dq, gq, w_uq, w_qr, w_dkv, w_kr, q_nope, q_rope, ckv, kr,
+                    ws, err, stream)
+
+    props = torch.cuda.get_device_properties(dev)
+    clock = ClockSampler(str(getattr(props, "uuid", "")), 0)
+    clock.start()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+        stream.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+    stream.synchronize()
+    clock.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())}")
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    esz = 2 if w.dtype == "bf16" else 4
+    weights = sum(int(t.numel()) for t in (w_dq, w_uq, w_qr, w_dkv, w_kr) if t is not None)
+    moved = (weights + x.numel() + q_nope.numel() + q_rope.numel() + ckv.numel() +
+             kr.numel()) * esz
+    flops = 2 * n * weights
+    hbm, _, _, src = load_peaks()
+    gbs = moved / (us * 1e-6) / 1e9
+    print(json.dumps({
+        "metric": "decode front end (mla_project): weight stream GB/s",
+        "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": f"{args.workload} front end: d_model={w.d_model} "
+                               f"q_rank={w.q_rank} H={H} d_h={dh} d_r={dr} r={r} tokens={n}",
+                   "l2": "weights larger than L2 (streamed every step)"},
+        "us_per_step": us, "algorithmic_bytes": moved, "algorithmic_flops": flops,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm, "peak_source": src},
+        "gpu_launches": (4 if w.q_rank else 2) * args.steps,
+        "clocks": clock.summary(t0, time.time(), "warm-up and timed steps"),
+    }), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     import mla_inputs as mi
 
+    if args.front:
+        return run_front(args, mi.WORKLOADS[args.workload])
     if args.context_parallel:
         return run_context_parallel(args)
     w = mi.WORKLOADS[args.workload]

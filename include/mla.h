@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 4
+#define MLA_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define MLA_API __attribute__((visibility("default")))
@@ -236,6 +236,45 @@ MLA_API mla_status mla_decode_step(const mla_config* cfg, const void* q_nope, co
                                    int32_t q_per_seq, void* q_work, void* workspace,
                                    size_t workspace_bytes, float* out_latent, float* lse,
                                    const void* w_uv, void* o, uint32_t* dev_err, void* stream);
+
+/*
+ * The decode front end: hidden states x -> the four per-token inputs of the calls above
+ * ([B] The MLAAttention module: c_q = RMSNorm(W_DQ x), q = W_UQ c_q; [D] the RoPE query and
+ * the shared RoPE key are projected from x; c_kv = W_DKV x, normalised at append).
+ */
+typedef struct {
+  int32_t d_model;  /* hidden size: the K of every product with x                          */
+  int32_t q_rank;   /* query latent width r_q; 0 for a full-rank query (q_nope = W_Q x)     */
+  float q_rms_eps;  /* eps of the RMSNorm of c_q                                            */
+} mla_front_config;
+
+/* Workspace of mla_project in bytes (0 for an invalid configuration); 256-byte aligned. */
+MLA_API size_t mla_project_workspace_size(const mla_config* cfg, const mla_front_config* front,
+                                          int32_t n_tokens);
+
+/*
+ * mla_project -- for n_tokens tokens x (n_tokens, d_model) dtype, with weights in the
+ * nn.Linear layout (out_features, d_model or q_rank) dtype:
+ *   q_rank > 0:  c_q = W_DQ x (w_dq: (q_rank, d_model)), c_q' = c_q / sqrt(mean(c_q^2) + eps)
+ *                * gamma_q (fp32 statistics; gamma_q (q_rank) float32), stored in dtype;
+ *                q_nope = W_UQ c_q' (w_uq: (H * d_h, q_rank));
+ *   q_rank == 0: q_nope = W_Q x (w_dq holds W_Q: (H * d_h, d_model)); gamma_q, w_uq unused;
+ *   q_rope = W_QR x (w_qr: (H * d_r, d_model)), ckv_raw = W_DKV x (w_dkv: (r, d_model)),
+ *   krope_raw = W_KR x (w_kr: (d_r, d_model)); with d_r == 0, w_qr, w_kr, q_rope and
+ *   krope_raw are unused.
+ * Outputs q_nope (n, H, d_h), q_rope (n, H, d_r), ckv_raw (n, r), krope_raw (n, d_r), dtype:
+ * the inputs of mla_absorb_query and mla_append_latent. Products accumulate in fp32 and are
+ * rounded once. bf16 with d_model and q_rank multiples of 8 runs on the tensor cores (x and
+ * every weight 16-byte aligned); fp32 on CUDA cores; bf16 with other widths returns
+ * MLA_ERR_UNSUPPORTED. Deterministic. q_rank at most
+ * 12288, d_model at most 57344. dev_err may be NULL (MLA_DEV_WAIT_TIMEOUT as elsewhere).
+ */
+MLA_API mla_status mla_project(const mla_config* cfg, const mla_front_config* front,
+                               const void* x, const void* w_dq, const float* gamma_q,
+                               const void* w_uq, const void* w_qr, const void* w_dkv,
+                               const void* w_kr, void* q_nope, void* q_rope, void* ckv_raw,
+                               void* krope_raw, int32_t n_tokens, void* workspace,
+                               size_t workspace_bytes, uint32_t* dev_err, void* stream);
 
 /* Most parts mla_combine_partials merges in one call. */
 #define MLA_MAX_COMBINE_PARTS 256

@@ -234,10 +234,14 @@ class LayerDraw:
     gamma_kv: np.ndarray           # (r,)  ones
 
 
-def layer_draw(w: Workload, seed: int = 0) -> LayerDraw:
-    """Hidden states N(0, 1) and nn.Linear-shaped weights N(0, 1/fan_in), float64."""
+def layer_draw(w: Workload, seed: int = 0, x_rows: Optional[int] = None) -> LayerDraw:
+    """Hidden states N(0, 1) and nn.Linear-shaped weights N(0, 1/fan_in), float64.
+
+    x is (B, longest sequence, d_model), or (x_rows, d_model) when x_rows is given (the
+    tokens of one step, for the front end alone).
+    """
     H, dh, r, dr, dm = w.num_heads, w.head_dim, w.kv_rank, w.rope_dim, w.d_model
-    rows = int(total_rows(w, seed).max())
+    x_shape = (w.batch, int(total_rows(w, seed).max()), dm) if x_rows is None else (x_rows, dm)
 
     def lin(stream, out_f, in_f):
         return _normal(seed, stream, (out_f, in_f), 1.0 / math.sqrt(in_f)).astype(np.float64)
@@ -250,7 +254,7 @@ def layer_draw(w: Workload, seed: int = 0) -> LayerDraw:
         w_uq = lin(_S_WUQ, H * dh, w.q_rank)
         gq = np.ones(w.q_rank)
     return LayerDraw(
-        x=_normal(seed, _S_X, (w.batch, rows, dm)).astype(np.float64),
+        x=_normal(seed, _S_X, x_shape).astype(np.float64),
         w_q=w_q, w_dq=w_dq, w_uq=w_uq,
         w_qr=lin(_S_WQR, H * dr, dm),
         w_dkv=lin(_S_WDKV, r, dm),

@@ -37,6 +37,10 @@ class MlaConfig(ctypes.Structure):
                 ("dtype", _c_i32), ("decode_kernel", _c_i32)]
 
 
+class MlaFrontConfig(ctypes.Structure):
+    _fields_ = [("d_model", _c_i32), ("q_rank", _c_i32), ("q_rms_eps", _c_f32)]
+
+
 class MlaError(RuntimeError):
     def __init__(self, status: int, where: str):
         super().__init__(f"{where}: {status_string(status)}")
@@ -65,6 +69,9 @@ def _load():
                                      _c_i32, _vp, _c_i32, _c_i32, _vp, _vp, _sz, _vp, _vp, _vp,
                                      _vp, _vp, _vp]),
         "mla_combine_partials": (_c_i32, [P, _vp, _vp, _c_i32, _c_i32, _vp, _vp, _vp]),
+        "mla_project_workspace_size": (_sz, [P, ctypes.POINTER(MlaFrontConfig), _c_i32]),
+        "mla_project": (_c_i32, [P, ctypes.POINTER(MlaFrontConfig), _vp, _vp, _vp, _vp, _vp,
+                                 _vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _vp, _sz, _vp, _vp]),
         "mla_status_string": (ctypes.c_char_p, [_c_i32]),
         "mla_abi_version": (_c_i32, []),
     }
@@ -225,6 +232,28 @@ def combine_partials(cfg: Config, part_latent, part_lse, out_latent, lse=None, s
                                     int(part_latent.shape[0]), int(part_latent.shape[1]),
                                     _ptr(out_latent), _ptr(lse), _stream(stream)),
            "mla_combine_partials")
+
+
+def front_config(d_model: int, q_rank: int = 0, q_rms_eps: float = 1e-6) -> MlaFrontConfig:
+    """mla_front_config: hidden size, query rank (0: full-rank query), RMSNorm eps of c_q."""
+    return MlaFrontConfig(d_model, q_rank, q_rms_eps)
+
+
+def project_workspace_size(cfg: Config, front: MlaFrontConfig, n_tokens: int) -> int:
+    return int(lib.mla_project_workspace_size(ctypes.byref(cfg.c()), ctypes.byref(front),
+                                              n_tokens))
+
+
+def project(cfg: Config, front: MlaFrontConfig, x, w_dq, gamma_q, w_uq, w_qr, w_dkv, w_kr,
+            q_nope, q_rope, ckv_raw, krope_raw, workspace, dev_err=None, stream=None):
+    """mla_project: hidden states x (n, d_model) -> q_nope, q_rope, ckv_raw, krope_raw."""
+    c = cfg.c()
+    _check(lib.mla_project(ctypes.byref(c), ctypes.byref(front), _ptr(x), _ptr(w_dq),
+                           _ptr(gamma_q), _ptr(w_uq), _ptr(w_qr), _ptr(w_dkv), _ptr(w_kr),
+                           _ptr(q_nope), _ptr(q_rope), _ptr(ckv_raw), _ptr(krope_raw),
+                           int(x.shape[0]), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _ptr(dev_err),
+                           _stream(stream)), "mla_project")
 
 
 def abi_version() -> int:

@@ -1,5 +1,6 @@
 // C ABI of libmla: argument validation, workspace carving and kernel dispatch.
 // Every entry point validates synchronously before any CUDA call and only enqueues work.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 
@@ -11,6 +12,14 @@ namespace mla {
 // decode_plan.cu: the merge behind mla_combine_partials
 cudaError_t launch_combine_parts(const float* part_o, const float* part_lse, int parts, int n,
                                  int H, int r, float* out, float* lse, cudaStream_t st);
+// front_tc.cu: the products behind mla_project
+bool front_tc_supported(const mla_config& c, int K);
+size_t front_part_bytes(const mla_config& c, int K, int n, const int* rows, int nseg,
+                        bool norm);
+cudaError_t launch_front_linear(const mla_config& c, const void* x, int n, int K,
+                                const void* const* w, const int* rows, void* const* out, int nseg,
+                                int norm_seg, const float* gamma, float eps, void* part,
+                                uint32_t* err, cudaStream_t st);
 }  // namespace mla
 
 namespace {
@@ -90,6 +99,103 @@ const char* mla_status_string(mla_status s) {
 }
 
 int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
+
+}  // extern "C"
+
+namespace {
+
+// Byte offsets of mla_project's workspace: the K-split partial sums (shared by the two
+// products, which run one after the other), then c_q' (n x q_rank, dtype).
+struct FrontLayout {
+  size_t part, cq, total;
+};
+
+bool front_valid(const mla_config* cfg, const mla_front_config* f, int32_t n) {
+  return valid_config(cfg) && f && f->d_model >= 1 && f->d_model <= 57344 && f->q_rank >= 0 &&
+         f->q_rank <= 12288 && std::isfinite(f->q_rms_eps) && f->q_rms_eps >= 0.f && n >= 0;
+}
+
+// Output rows of the products with x, in launch order: c_q (or q_nope), q_rope, c_kv, k_rope
+// (the RoPE ones only when d_r > 0). Returns their count.
+int front_rows(const mla_config& c, const mla_front_config& f, int* rows) {
+  int nseg = 0;
+  rows[nseg++] = f.q_rank > 0 ? f.q_rank : c.num_heads * c.head_dim;
+  if (c.rope_dim > 0) rows[nseg++] = c.num_heads * c.rope_dim;
+  rows[nseg++] = c.kv_rank;
+  if (c.rope_dim > 0) rows[nseg++] = c.rope_dim;
+  return nseg;
+}
+
+FrontLayout front_layout(const mla_config& c, const mla_front_config& f, int n) {
+  int rows1[4];
+  const int nseg = front_rows(c, f, rows1);
+  size_t part = front_part_bytes(c, f.d_model, n, rows1, nseg, f.q_rank > 0);
+  if (f.q_rank > 0) {
+    const int rows3[1] = {c.num_heads * c.head_dim};
+    part = std::max(part, front_part_bytes(c, f.q_rank, n, rows3, 1, false));
+  }
+  FrontLayout L;
+  L.part = 0;
+  L.cq = (part + 255) / 256 * 256;
+  const size_t esz = c.dtype == MLA_BF16 ? 2 : 4;
+  L.total = L.cq + ((size_t)n * f.q_rank * esz + 255) / 256 * 256;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mla_project_workspace_size(const mla_config* cfg, const mla_front_config* front,
+                                  int32_t n_tokens) {
+  if (!front_valid(cfg, front, n_tokens) || n_tokens == 0) return 0;
+  return front_layout(*cfg, *front, n_tokens).total;
+}
+
+mla_status mla_project(const mla_config* cfg, const mla_front_config* front, const void* x,
+                       const void* w_dq, const float* gamma_q, const void* w_uq,
+                       const void* w_qr, const void* w_dkv, const void* w_kr, void* q_nope,
+                       void* q_rope, void* ckv_raw, void* krope_raw, int32_t n_tokens,
+                       void* workspace, size_t workspace_bytes, uint32_t* dev_err,
+                       void* stream) {
+  if (!front_valid(cfg, front, n_tokens)) return MLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MLA_OK;
+  const mla_config& c = *cfg;
+  const mla_front_config& f = *front;
+  const bool rope = c.rope_dim > 0, low = f.q_rank > 0;
+  if (!x || !w_dq || !w_dkv || !q_nope || !ckv_raw || !workspace) return MLA_ERR_INVALID_ARG;
+  if (low && (!w_uq || !gamma_q)) return MLA_ERR_INVALID_ARG;
+  if (rope && (!w_qr || !w_kr || !q_rope || !krope_raw)) return MLA_ERR_INVALID_ARG;
+  const FrontLayout L = front_layout(c, f, n_tokens);
+  if (workspace_bytes < L.total || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+  if (c.dtype == MLA_BF16) {
+    if (!front_tc_supported(c, f.d_model) || (low && !front_tc_supported(c, f.q_rank)))
+      return MLA_ERR_UNSUPPORTED;
+    const void* ptrs[] = {x, w_dq, w_uq, w_qr, w_dkv, w_kr};
+    for (const void* p : ptrs)
+      if (p && !aligned(p, 16)) return MLA_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  const int H = c.num_heads, dh = c.head_dim;
+  uint8_t* ws = (uint8_t*)workspace;
+  void* cq = ws + L.cq;
+  // the products with x: c_q (or q_nope), q_rope, c_kv, k_rope in one launch
+  int rows1[4];
+  const int nseg = front_rows(c, f, rows1);
+  const void* w1[4] = {w_dq, rope ? w_qr : w_dkv, w_dkv, w_kr};
+  void* out1[4] = {low ? cq : q_nope, rope ? q_rope : ckv_raw, ckv_raw, krope_raw};
+  cudaError_t e = launch_front_linear(c, x, n_tokens, f.d_model, w1, rows1, out1, nseg,
+                                      low ? 0 : -1, gamma_q, f.q_rms_eps, ws + L.part, dev_err,
+                                      st);
+  if (e == cudaSuccess && low) {
+    const void* w3[1] = {w_uq};
+    const int rows3[1] = {H * dh};
+    void* out3[1] = {q_nope};
+    e = launch_front_linear(c, cq, n_tokens, f.q_rank, w3, rows3, out3, 1, -1, nullptr, 0.f,
+                            ws + L.part, dev_err, st);
+  }
+  return from_cuda(e);
+}
 
 mla_status mla_combine_partials(const mla_config* cfg, const float* part_latent,
                                 const float* part_lse, int32_t parts, int32_t n,
