@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-kernel", default="auto", choices=["auto", "simt", "tensor"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill", type=int, nargs=2, default=None, metavar=("B", "S"),
+                    help="time mla_prefill on B prompts of S tokens at the workload's head shape")
     ap.add_argument("--front", action="store_true",
                     help="time the decode front end (mla_project) at the workload's shape")
     ap.add_argument("--context-parallel", type=int, default=0, metavar="G",
@@ -797,10 +799,91 @@ def run_front(args, w):
     return 0
 
 
+# ---------------------------------------------------------------------------------------
+# Prefill (mla_prefill): B prompts of S tokens, causal, in the expanded form. FLOPs counted:
+# the K and V expansion (2 n r H (d_h + d_v)) and the attention over the causal half
+# (2 H (d_h + d_r + d_v) per visible (query, key) pair).
+# ---------------------------------------------------------------------------------------
+def run_prefill(args, w):
+    import torch
+
+    import mla_latent_kv_44_b200 as mla
+
+    rank, world, local = dist_env()
+    if world > 1:
+        if rank == 0:
+            print(json.dumps({"metric": "prefill", "unavailable":
+                              "measured on one GPU; run without torchrun"}))
+        return 0
+    B, S = args.prefill
+    dev = torch.device("cuda", 0)
+    H, dh, dr, dv, r = w.num_heads, w.head_dim, w.rope_dim, w.head_dim_v, w.kv_rank
+    cfg = mla.Config(num_heads=H, head_dim=dh, kv_rank=r, rope_dim=dr, block_size=64,
+                     dtype=w.dtype)
+    tdt = cfg.torch_dtype
+    n = B * S
+    gen = torch.Generator(device=dev).manual_seed(1234)
+
+    def draw(*shape, std=1.0):
+        return (torch.randn(*shape, generator=gen, device=dev) * std).to(tdt)
+
+    q_nope, q_rope = draw(n, H, dh), draw(n, H, dr)
+    rows = draw(n, r + dr)
+    w_uk, w_uv = draw(H, dh, r, std=r ** -0.5), draw(H, dv, r, std=r ** -0.5)
+    pos = torch.arange(S, dtype=torch.int32, device=dev).repeat(B)
+    cu = torch.arange(0, n + 1, S, dtype=torch.int32, device=dev)
+    o = torch.empty((n, H, dv), dtype=tdt, device=dev)
+    ws = torch.empty(mla.prefill_workspace_size(cfg, n), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        mla.prefill(cfg, q_nope, q_rope, pos, rows, w_uk, w_uv, cu, S, o, ws, err, stream)
+
+    props = torch.cuda.get_device_properties(dev)
+    clock = ClockSampler(str(getattr(props, "uuid", "")), 0)
+    clock.start()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+        stream.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+    stream.synchronize()
+    clock.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())}")
+    ms = e0.elapsed_time(e1) / args.steps
+    pairs = B * S * (S + 1) // 2
+    flops = 2 * n * r * H * (dh + dv) + 2 * H * (dh + dr + dv) * pairs
+    tflops = flops / (ms * 1e-3) / 1e12
+    _, peak, _, src = load_peaks()
+    print(json.dumps({
+        "metric": "MLA prefill TFLOP/s (causal, expanded form)", "value": tflops,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "dtype": w.dtype, "data": "synthetic (seeded N(0,1))",
+        "config": {"workload": f"{args.workload} heads: H={H} d_h={dh} d_r={dr} d_v={dv} "
+                               f"r={r}, {B} prompts x {S} tokens"},
+        "ms_per_step": ms, "tokens_per_s": n / (ms * 1e-3), "algorithmic_flops": flops,
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "peak_source": src},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clock.summary(t0, time.time(), "warm-up and timed steps"),
+    }), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     import mla_inputs as mi
 
+    if args.prefill:
+        return run_prefill(args, mi.WORKLOADS[args.workload])
     if args.front:
         return run_front(args, mi.WORKLOADS[args.workload])
     if args.context_parallel:

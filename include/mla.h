@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 5
+#define MLA_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define MLA_API __attribute__((visibility("default")))
@@ -274,6 +274,32 @@ MLA_API mla_status mla_project(const mla_config* cfg, const mla_front_config* fr
                                const void* w_uq, const void* w_qr, const void* w_dkv,
                                const void* w_kr, void* q_nope, void* q_rope, void* ckv_raw,
                                void* krope_raw, int32_t n_tokens, void* workspace,
+                               size_t workspace_bytes, uint32_t* dev_err, void* stream);
+
+/* Workspace of mla_prefill in bytes (0 for an invalid configuration); 256-byte aligned. */
+MLA_API size_t mla_prefill_workspace_size(const mla_config* cfg, int32_t n_tokens);
+
+/*
+ * mla_prefill -- causal self-attention of prompts in the expanded form ([B] The MLAAttention
+ * module: K and V rebuilt from every cached latent, the causal mask when S > 1; the expanded
+ * form takes d_h + d_r multiply-adds per score against r + d_r absorbed, so it is the cheaper
+ * one when every key serves many queries). For a batch of prompts packed one after another
+ * (sequence b holds tokens cu_seqlens[b] .. cu_seqlens[b + 1] - 1) and every head h:
+ *   K[j, h] = [W_UK[h] c_kv[j] ‖ k_rope[j]],  V[j, h] = W_UV[h] c_kv[j],
+ *   Q[i, h] = [q_nope[i, h] ‖ RoPE(q_rope[i, h], pos[i])],
+ *   o[i, h] = sum_j p_j V[j, h],  p = softmax_j(softmax_scale * Q[i, h] . K[j, h])
+ * over the keys j of i's sequence with j <= i.
+ * q_nope (n, H, d_h), q_rope (n, H, d_r) before rotation, pos (n) int32, rows (n, r + d_r):
+ * the tokens' cache rows [RMSNorm(c_kv) * gamma ‖ RoPE(k_rope)] as mla_append_latent writes
+ * them, here contiguous; w_uk (H, d_h, r), w_uv (H, d_v, r); cu_seqlens (batch + 1) int32 on
+ * the device, non-decreasing from 0 to n; max_seqlen >= every sequence's length (host value);
+ * o (n, H, d_v). All dtype. bf16 with d_h = d_v = 128, d_r = 64 runs on the tensor cores
+ * (every pointer 16-byte aligned); other shapes and fp32 on CUDA cores (d_v <= 256).
+ */
+MLA_API mla_status mla_prefill(const mla_config* cfg, const void* q_nope, const void* q_rope,
+                               const int32_t* pos, const void* rows, const void* w_uk,
+                               const void* w_uv, const int32_t* cu_seqlens, int32_t batch,
+                               int32_t max_seqlen, int32_t n_tokens, void* o, void* workspace,
                                size_t workspace_bytes, uint32_t* dev_err, void* stream);
 
 /* Most parts mla_combine_partials merges in one call. */

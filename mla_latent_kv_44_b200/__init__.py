@@ -69,6 +69,9 @@ def _load():
                                      _c_i32, _vp, _c_i32, _c_i32, _vp, _vp, _sz, _vp, _vp, _vp,
                                      _vp, _vp, _vp]),
         "mla_combine_partials": (_c_i32, [P, _vp, _vp, _c_i32, _c_i32, _vp, _vp, _vp]),
+        "mla_prefill_workspace_size": (_sz, [P, _c_i32]),
+        "mla_prefill": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _c_i32,
+                                 _vp, _vp, _sz, _vp, _vp]),
         "mla_project_workspace_size": (_sz, [P, ctypes.POINTER(MlaFrontConfig), _c_i32]),
         "mla_project": (_c_i32, [P, ctypes.POINTER(MlaFrontConfig), _vp, _vp, _vp, _vp, _vp,
                                  _vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _vp, _sz, _vp, _vp]),
@@ -254,6 +257,21 @@ def project(cfg: Config, front: MlaFrontConfig, x, w_dq, gamma_q, w_uq, w_qr, w_
                            int(x.shape[0]), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _ptr(dev_err),
                            _stream(stream)), "mla_project")
+
+
+def prefill_workspace_size(cfg: Config, n_tokens: int) -> int:
+    return int(lib.mla_prefill_workspace_size(ctypes.byref(cfg.c()), n_tokens))
+
+
+def prefill(cfg: Config, q_nope, q_rope, pos, rows, w_uk, w_uv, cu_seqlens, max_seqlen: int, o,
+            workspace, dev_err=None, stream=None):
+    """mla_prefill: causal attention of packed prompts (cu_seqlens: batch + 1 offsets)."""
+    c = cfg.c()
+    _check(lib.mla_prefill(ctypes.byref(c), _ptr(q_nope), _ptr(q_rope), _ptr(pos), _ptr(rows),
+                           _ptr(w_uk), _ptr(w_uv), _ptr(cu_seqlens), int(cu_seqlens.shape[0]) - 1,
+                           int(max_seqlen), int(q_nope.shape[0]), _ptr(o), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _ptr(dev_err),
+                           _stream(stream)), "mla_prefill")
 
 
 def abi_version() -> int:

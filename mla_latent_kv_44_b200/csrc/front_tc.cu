@@ -47,7 +47,7 @@ struct FrontSeg {
 struct LinearArgs {
   FrontSeg seg[kFrontMaxSegs];
   const float* wf[kFrontMaxSegs];  // fp32 weights (CUDA-core kernel only)
-  int nseg, n, K, splits, ntile;
+  int nseg, n, K, ldx, splits, ntile;  // ldx: elements between consecutive rows of x
   uint32_t* err;
 };
 
@@ -215,7 +215,7 @@ linear_simt_kernel(const float* x, const LinearArgs a) {
   wait_prior_grid();
   for (int t = blockIdx.z; t < a.n; t += gridDim.z) {
     __syncthreads();
-    for (int k = threadIdx.x; k < a.K; k += blockDim.x) xs[k] = x[(size_t)t * a.K + k];
+    for (int k = threadIdx.x; k < a.K; k += blockDim.x) xs[k] = x[(size_t)t * a.ldx + k];
     __syncthreads();
     if (row < sg.rows) {
       const float* wr = a.wf[s] + (size_t)row * a.K;
@@ -352,9 +352,10 @@ size_t front_part_bytes(const mla_config& c, int K, int n, const int* rows, int 
 }
 
 // y_s = W_s x for up to four weights W_s (rows[s] x K, nn.Linear layout) sharing the input
-// x (n x K); outputs in the config's dtype at out[s] (n x rows[s]); segment norm_seg (or -1)
-// is RMS-normalised with gain gamma. `part` holds front_part_bytes(...).
-cudaError_t launch_front_linear(const mla_config& c, const void* x, int n, int K,
+// x (n rows of K values, ldx elements apart); outputs in the config's dtype at out[s]
+// (n x rows[s]); segment norm_seg (or -1) is RMS-normalised with gain gamma. `part` holds
+// front_part_bytes(...).
+cudaError_t launch_front_linear(const mla_config& c, const void* x, int n, int K, int ldx,
                                 const void* const* w, const int* rows, void* const* out, int nseg,
                                 int norm_seg, const float* gamma, float eps, void* part,
                                 uint32_t* err, cudaStream_t st) {
@@ -387,6 +388,7 @@ cudaError_t launch_front_linear(const mla_config& c, const void* x, int n, int K
   a.nseg = nseg;
   a.n = n;
   a.K = K;
+  a.ldx = ldx;
   a.splits = splits;
   a.ntile = ntile;
   a.err = err;
@@ -399,7 +401,7 @@ cudaError_t launch_front_linear(const mla_config& c, const void* x, int n, int K
                          kFrontRows))
         return cudaErrorInvalidValue;
     }
-    if (!make_bf16_map(&tx, x, (uint64_t)K, (uint64_t)n, (uint64_t)K * 2, (uint32_t)ntile))
+    if (!make_bf16_map(&tx, x, (uint64_t)K, (uint64_t)n, (uint64_t)ldx * 2, (uint32_t)ntile))
       return cudaErrorInvalidValue;
     const size_t smem = front_smem(ntile);
     e = cudaFuncSetAttribute(linear_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

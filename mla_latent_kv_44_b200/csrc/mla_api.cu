@@ -16,10 +16,17 @@ cudaError_t launch_combine_parts(const float* part_o, const float* part_lse, int
 bool front_tc_supported(const mla_config& c, int K);
 size_t front_part_bytes(const mla_config& c, int K, int n, const int* rows, int nseg,
                         bool norm);
-cudaError_t launch_front_linear(const mla_config& c, const void* x, int n, int K,
+cudaError_t launch_front_linear(const mla_config& c, const void* x, int n, int K, int ldx,
                                 const void* const* w, const int* rows, void* const* out, int nseg,
                                 int norm_seg, const float* gamma, float eps, void* part,
                                 uint32_t* err, cudaStream_t st);
+// prefill_tc.cu: mla_prefill
+bool prefill_tc_supported(const mla_config& c);
+size_t prefill_workspace_bytes(const mla_config& c, int n);
+cudaError_t launch_prefill(const mla_config& c, const void* q_nope, const void* q_rope,
+                           const int32_t* pos, const void* rows, const void* w_uk,
+                           const void* w_uv, const int32_t* cu, int batch, int max_seqlen, int n,
+                           void* o, void* ws, uint32_t* err, cudaStream_t st);
 }  // namespace mla
 
 namespace {
@@ -184,17 +191,54 @@ mla_status mla_project(const mla_config* cfg, const mla_front_config* front, con
   const int nseg = front_rows(c, f, rows1);
   const void* w1[4] = {w_dq, rope ? w_qr : w_dkv, w_dkv, w_kr};
   void* out1[4] = {low ? cq : q_nope, rope ? q_rope : ckv_raw, ckv_raw, krope_raw};
-  cudaError_t e = launch_front_linear(c, x, n_tokens, f.d_model, w1, rows1, out1, nseg,
+  cudaError_t e = launch_front_linear(c, x, n_tokens, f.d_model, f.d_model, w1, rows1, out1, nseg,
                                       low ? 0 : -1, gamma_q, f.q_rms_eps, ws + L.part, dev_err,
                                       st);
   if (e == cudaSuccess && low) {
     const void* w3[1] = {w_uq};
     const int rows3[1] = {H * dh};
     void* out3[1] = {q_nope};
-    e = launch_front_linear(c, cq, n_tokens, f.q_rank, w3, rows3, out3, 1, -1, nullptr, 0.f,
-                            ws + L.part, dev_err, st);
+    e = launch_front_linear(c, cq, n_tokens, f.q_rank, f.q_rank, w3, rows3, out3, 1, -1,
+                            nullptr, 0.f, ws + L.part, dev_err, st);
   }
   return from_cuda(e);
+}
+
+size_t mla_prefill_workspace_size(const mla_config* cfg, int32_t n_tokens) {
+  if (!valid_config(cfg) || n_tokens < 1) return 0;
+  return prefill_workspace_bytes(*cfg, n_tokens);
+}
+
+mla_status mla_prefill(const mla_config* cfg, const void* q_nope, const void* q_rope,
+                       const int32_t* pos, const void* rows, const void* w_uk, const void* w_uv,
+                       const int32_t* cu_seqlens, int32_t batch, int32_t max_seqlen,
+                       int32_t n_tokens, void* o, void* workspace, size_t workspace_bytes,
+                       uint32_t* dev_err, void* stream) {
+  if (!valid_config(cfg) || batch < 0 || n_tokens < 0 || max_seqlen < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (batch == 0 || n_tokens == 0) return MLA_OK;
+  const mla_config& c = *cfg;
+  const bool rope = c.rope_dim > 0;
+  if (!q_nope || (rope && (!q_rope || !pos)) || !rows || !w_uk || !w_uv || !cu_seqlens || !o ||
+      !workspace || max_seqlen < 1)
+    return MLA_ERR_INVALID_ARG;
+  // d_v: a warp's values on CUDA cores; d_h, d_r: the query is packed in 16-byte pieces
+  const int vec = c.dtype == MLA_BF16 ? 8 : 4;
+  if (c.head_dim_v > 256 || c.head_dim % vec != 0 || c.rope_dim % vec != 0)
+    return MLA_ERR_UNSUPPORTED;
+  if (!aligned(q_nope, 16) || (rope && !aligned(q_rope, 16))) return MLA_ERR_INVALID_ARG;
+  if (workspace_bytes < prefill_workspace_bytes(c, n_tokens) || !aligned(workspace, 256))
+    return MLA_ERR_WORKSPACE;
+  if (c.dtype == MLA_BF16) {
+    // the expansion of K and V streams the weights on the tensor cores (16-byte rows)
+    if (c.kv_rank % 8 != 0 || (c.kv_rank + c.rope_dim) % 8 != 0) return MLA_ERR_UNSUPPORTED;
+    const void* ptrs[] = {q_nope, q_rope, rows, w_uk, w_uv, o};
+    for (const void* p : ptrs)
+      if (p && !aligned(p, 16)) return MLA_ERR_INVALID_ARG;
+  }
+  return from_cuda(launch_prefill(c, q_nope, q_rope, pos, rows, w_uk, w_uv, cu_seqlens, batch,
+                                  max_seqlen, n_tokens, o, workspace, dev_err,
+                                  (cudaStream_t)stream));
 }
 
 mla_status mla_combine_partials(const mla_config* cfg, const float* part_latent,

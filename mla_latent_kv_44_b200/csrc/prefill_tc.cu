@@ -1,0 +1,458 @@
+// MLA prefill: causal attention of a prompt's tokens over themselves, in the expanded form,
+// for sm_100a.
+//   K_nope[j, h] = W_UK[h] c_kv[j],  V[j, h] = W_UV[h] c_kv[j]           ("MLA from scratch in
+//   s = scale * ([q_nope ‖ RoPE(q_rope)] . [K_nope ‖ k_rope]),            PyTorch", The
+//   query i attends keys 0 .. i of its sequence, o = softmax(s) V          MLAAttention module:
+//                                                                         K and V rebuilt from
+// the latent, the causal mask over the S > 1 new tokens). With many queries per key the
+// expanded form costs fewer FLOPs than the absorbed one (d_h + d_r = 192 per score against
+// r + d_r = 576), so K and V are expanded once per key: one split-K weight-stream launch of the
+// front end's kernel (W_UK and W_UV as two segments, c_kv read in place from the cache rows).
+// A pack kernel writes the query as [q_nope ‖ RoPE(q_rope)] (angles in double).
+// The attention kernel takes one CTA per (128-query tile, head) of a sequence (DeepSeek-V2's
+// head shape: d_h = 128, d_r = 64, d_v = 128, bf16): the query tile stays in shared memory;
+// per 128-key tile, TMA brings the key tile (K_nope of the head and the shared k_rope: three
+// 64-wide slabs) and the value tile, one thread issues S = Q K^T (M = 128 queries, N = 128
+// keys, 12 K-steps) into TMEM, the four warps (a thread per query row) take the row maximum,
+// rescale O in TMEM when the maximum grows by more than 2^8 (exp2 units), write P in bf16 into
+// shared memory as the A operand, and one thread issues O += P V (N = 128, V MN-major). Tiles
+// above the diagonal are skipped; the diagonal tile is masked. Other shapes and fp32 take a
+// CUDA-core kernel (a warp per (query, head), online softmax over the keys).
+// Every mbarrier wait gives up after 1 s: the kernel then sets MLA_DEV_WAIT_TIMEOUT, waits
+// (bounded) for what it issued, frees TMEM and returns.
+#include <algorithm>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+#include "tma_map.h"
+
+namespace mla {
+
+size_t front_part_bytes(const mla_config& c, int K, int n, const int* rows, int nseg,
+                        bool norm);
+cudaError_t launch_front_linear(const mla_config& c, const void* x, int n, int K, int ldx,
+                                const void* const* w, const int* rows, void* const* out, int nseg,
+                                int norm_seg, const float* gamma, float eps, void* part,
+                                uint32_t* err, cudaStream_t st);
+
+namespace {
+
+constexpr unsigned long long kPfTimeoutNs = 1000000000ull;
+constexpr int kPfTile = 128;                   // queries per CTA = keys per tile
+constexpr int kPfSlabBytes = kPfTile * 128;    // 128 rows x 64 bf16: 16 KB
+constexpr int kPfQ = 0;                        // query: 3 slabs (q_nope 0-63, 64-127, q_rope)
+constexpr int kPfK = kPfQ + 3 * kPfSlabBytes;  // keys: 3 slabs (K_nope 0-63, 64-127, k_rope)
+constexpr int kPfV = kPfK + 3 * kPfSlabBytes;  // values: 2 slabs (d_v 0-63, 64-127), MN-major
+constexpr int kPfP = kPfV + 2 * kPfSlabBytes;  // P: 2 slabs (keys 0-63, 64-127), K-major
+constexpr int kPfBar = kPfP + 2 * kPfSlabBytes;
+constexpr int kPfSmem = kPfBar + 64 + 1024;
+constexpr uint32_t kPfTmemCols = 256;          // S: columns 0-127, O: 128-255
+
+__device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try(bar, parity)) {
+    if (globaltimer() - t0 > kPfTimeoutNs) {
+      set_error(err, MLA_DEV_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// The sequence of token index i: cu_seqlens[b] <= i < cu_seqlens[b + 1] (binary search).
+__device__ __forceinline__ int seq_of(const int32_t* cu, int batch, int i) {
+  int lo = 0, hi = batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cu[mid] <= i) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// Q = [q_nope ‖ RoPE(q_rope, pos)] per (token, head): grid (tokens), 16-byte pieces (VEC
+// values) per thread: q_nope pieces copied, q_rope pieces rotated pair by pair (angle and
+// rotation in double, rounded once).
+template <typename T>
+__global__ void __launch_bounds__(256)
+prefill_pack_kernel(const T* q_nope, const T* q_rope, const int32_t* pos, T* q, int H, int dh,
+                    int dr, float base) {
+  constexpr int VEC = 16 / sizeof(T);
+  extern __shared__ double cs[];  // [2][dr / 2]: cos, sin of the token's angles
+  const int n = blockIdx.x, half = dr / 2, D = dh + dr;
+  const int pn = dh / VEC, pr = dr / VEC, pd = pn + pr;  // pieces per head
+  wait_prior_grid();
+  for (int i = threadIdx.x; i < half; i += blockDim.x)
+    rope_cos_sin(pos[n], i, dr, base, &cs[i], &cs[half + i]);
+  __syncthreads();
+  for (int e = threadIdx.x; e < H * pd; e += blockDim.x) {
+    const int h = e / pd, c = e - h * pd;
+    uint4 out;
+    if (c < pn) {
+      out = *(const uint4*)(q_nope + ((size_t)n * H + h) * dh + c * VEC);
+    } else {
+      const int k0 = (c - pn) * VEC;  // first rope value of the piece (even)
+      const uint4 in = *(const uint4*)(q_rope + ((size_t)n * H + h) * dr + k0);
+      const T* x = (const T*)&in;
+      T* y = (T*)&out;
+#pragma unroll
+      for (int u = 0; u < VEC; u += 2) {
+        const int i = (k0 + u) >> 1;
+        const double x0 = to_f32(x[u]), x1 = to_f32(x[u + 1]);
+        y[u] = from_f32<T>((float)(x0 * cs[i] - x1 * cs[half + i]));
+        y[u + 1] = from_f32<T>((float)(x0 * cs[half + i] + x1 * cs[i]));
+      }
+    }
+    *(uint4*)(q + ((size_t)n * H + h) * D + c * VEC) = out;
+  }
+}
+
+struct PrefillArgs {
+  const int32_t* cu;
+  __nv_bfloat16* o;
+  uint32_t* err;
+  int batch, H, qtiles;  // qtiles: query tiles per sequence in the grid (max_seqlen / 128)
+  float c2;              // softmax scale * log2(e)
+};
+
+// Grid (batch * qtiles, H); 128 threads. TMA maps: q (n, H * 192), kn (n, H * 128),
+// rows (n, r + 64): k_rope at column r, v (n, H * 128); all with 128-row boxes of 64 columns.
+__global__ void __launch_bounds__(128)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kn,
+                  const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_v,
+                  const PrefillArgs a, int r) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sb = saddr(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x / a.qtiles, qt = blockIdx.x - b * a.qtiles, h = blockIdx.y;
+  const uint32_t bar_q = sb + kPfBar, bar_k = bar_q + 8, bar_v = bar_q + 16;
+  const uint32_t bar_s = bar_q + 24, bar_o = bar_q + 32;
+  uint32_t* tmem_slot = (uint32_t*)(smem + kPfBar + 40);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 5; ++i) mbar_init(bar_q + 8 * i, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     saddr(tmem_slot)),
+                 "r"(kPfTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  const uint32_t tmem = *tmem_slot;
+  wait_prior_grid();
+  const int start = a.cu[b], len = a.cu[b + 1] - start;
+  const int q0 = qt * kPfTile;
+  bool ok = true;
+  int issued_k = 0, issued_v = 0, done_s = 0, done_o = 0;  // phases, for the abort drain
+  if (q0 < len) {
+    const int nkt = (min(len, q0 + kPfTile) - 1) / kPfTile + 1;  // key tiles 0 .. diagonal
+    auto load_k = [&](int j) {
+      mbar_expect_tx(bar_k, 3 * kPfSlabBytes);
+      for (int s = 0; s < 2; ++s)
+        tma_load(sb + kPfK + s * kPfSlabBytes, &tm_kn, bar_k, h * 128 + 64 * s,
+                 start + j * kPfTile);
+      tma_load(sb + kPfK + 2 * kPfSlabBytes, &tm_kr, bar_k, r, start + j * kPfTile);
+    };
+    auto load_v = [&](int j) {
+      mbar_expect_tx(bar_v, 2 * kPfSlabBytes);
+      for (int s = 0; s < 2; ++s)
+        tma_load(sb + kPfV + s * kPfSlabBytes, &tm_v, bar_v, h * 128 + 64 * s,
+                 start + j * kPfTile);
+    };
+    if (threadIdx.x == 0) {
+      mbar_expect_tx(bar_q, 3 * kPfSlabBytes);
+      for (int s = 0; s < 3; ++s)
+        tma_load(sb + kPfQ + s * kPfSlabBytes, &tm_q, bar_q, h * 192 + 64 * s, start + q0);
+      load_k(0);
+      load_v(0);
+    }
+    issued_k = issued_v = 1;
+    const int qi = q0 + threadIdx.x;  // this thread's query (TMEM lane threadIdx.x)
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const uint32_t t_s = tmem + lane_base, t_o = tmem + lane_base + 128;
+    float m_ref = 0.f, l = 0.f;
+    if (threadIdx.x == 0) ok = pf_wait(bar_q, 0, a.err);
+    ok = __syncthreads_and(ok);
+    for (int j = 0; j < nkt && ok; ++j) {
+      // S = Q K_j^T
+      if (threadIdx.x == 0) {
+        ok = pf_wait(bar_k, j & 1, a.err);
+        if (ok) {
+          tc_after();
+          const uint32_t id = idesc(128, 128, 0, 0);
+          for (int ks = 0; ks < 12; ++ks) {
+            const uint32_t off = (uint32_t)(ks >> 2) * kPfSlabBytes + 32u * (uint32_t)(ks & 3);
+            mma_ss(tmem, sdesc(sb + kPfQ + off, 16, 1024, 2), sdesc(sb + kPfK + off, 16, 1024, 2),
+                   id, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(bar_s);
+        }
+      }
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
+      ok = pf_wait(bar_s, j & 1, a.err);
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
+      done_s = j + 1;
+      tc_after();
+      // the key buffer is free: the next tile's keys load during this tile's softmax and P . V
+      if (threadIdx.x == 0 && j + 1 < nkt) load_k(j + 1);
+      if (j + 1 < nkt) issued_k = j + 2;
+      uint32_t v[128];
+      tmem_ld128(t_s, v);
+      // causal mask: key k0 + c is visible to query qi when k0 + c <= qi (and inside the
+      // sequence, which qi < len implies)
+      const int k0 = j * kPfTile;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        const float s = (k0 + c <= qi) ? __uint_as_float(v[c]) * a.c2 : -INFINITY;
+        v[c] = __float_as_uint(s);
+        mx = fmaxf(mx, s);
+      }
+      float alpha = 1.f;
+      if (j == 0) {
+        m_ref = qi < len ? mx : 0.f;  // key 0 is always visible to a query of the sequence
+      } else if (mx > m_ref + 8.f) {
+        alpha = ex2(m_ref - mx);
+        m_ref = mx;
+      }
+      // P in bf16 as the A operand of P . V: row qi, keys in 2 slabs of 64 (128-byte rows
+      // swizzled by row % 8); l sums the bf16 values the MMA consumes
+      float rs = 0.f;
+      const uint32_t prow = sb + kPfP + (uint32_t)threadIdx.x * 128;
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 64 * s + 8 * g + 2 * e;
+            const float p0 = ex2(__uint_as_float(v[c]) - m_ref);
+            const float p1 = ex2(__uint_as_float(v[c + 1]) - m_ref);
+            w4[e] = pack_bf16(p0, p1);
+            rs += __uint_as_float(w4[e] << 16) + __uint_as_float(w4[e] & 0xffff0000u);
+          }
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           prow + s * kPfSlabBytes + 16u * (uint32_t)(g ^ (threadIdx.x & 7))),
+                       "r"(w4[0]), "r"(w4[1]), "r"(w4[2]), "r"(w4[3])
+                       : "memory");
+        }
+      }
+      l = l * alpha + rs;
+      // TMEM loads and stores are warp-wide: a warp rescales when any of its rows must
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // the previous P . V is complete (waited for below): rescale this row of O
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c0, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(t_o + c0, o);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async();
+      tc_before();
+      __syncthreads();
+      // O += P V_j
+      if (threadIdx.x == 0) {
+        ok = pf_wait(bar_v, j & 1, a.err);
+        if (ok) {
+          tc_after();
+          const uint32_t id = idesc(128, 128, 1);
+          for (int ks = 0; ks < 8; ++ks)  // 16 keys per step; V's two d_v slabs LBO apart
+            mma_ss(tmem + 128, sdesc(sb + kPfP + (uint32_t)(ks >> 2) * kPfSlabBytes + 32u * (ks & 3), 16, 1024, 2),
+                   sdesc(sb + kPfV + 2048u * (uint32_t)ks, kPfSlabBytes, 1024, 2), id,
+                   (j > 0 || ks > 0) ? 1u : 0u);
+          tc_commit(bar_o);
+        }
+      }
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
+      ok = __syncthreads_and(pf_wait(bar_o, j & 1, a.err));
+      if (!ok) break;
+      done_o = j + 1;
+      // values and P are free again
+      if (threadIdx.x == 0 && j + 1 < nkt) load_v(j + 1);
+      if (j + 1 < nkt) issued_v = j + 2;
+    }
+    if (ok) {
+      tc_after();
+      // o = O / l for this thread's query row, bf16 (every lane takes part in the warp-wide
+      // TMEM loads; rows past the sequence end store nothing)
+      const float inv = qi < len ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = a.o + ((size_t)(start + min(qi, len - 1)) * a.H + h) * 128;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(t_o + c0, o);
+        if (qi < len) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+            w.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+            w.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+            w.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+            *(uint4*)(dst + c0 + i) = w;
+          }
+        }
+      }
+    }
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  if (!ok && threadIdx.x == 0) {
+    // copies that may still land, MMAs that may still run
+    const uint64_t t0 = globaltimer();
+    while (issued_k > done_s && !mbar_try(bar_k, (issued_k - 1) & 1) &&
+           globaltimer() - t0 < kPfTimeoutNs) {
+    }
+    while (issued_v > done_o && !mbar_try(bar_v, (issued_v - 1) & 1) &&
+           globaltimer() - t0 < 2 * kPfTimeoutNs) {
+    }
+    tc_commit(bar_s);  // completes once every MMA issued so far is done
+    while (!mbar_try(bar_s, done_s & 1) && globaltimer() - t0 < 3 * kPfTimeoutNs) {
+    }
+  }
+  __syncthreads();
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kPfTmemCols)
+                 : "memory");
+}
+
+// CUDA-core prefill: a warp per (query, head); lanes split the score's dims and the value's.
+template <typename T>
+__global__ void __launch_bounds__(128)
+prefill_simt_kernel(const T* q, const T* kn, const T* rows, const T* v, const int32_t* cu,
+                    int batch, int H, int dh, int dr, int dv, int ldr, int r, float c2, T* o) {
+  const int i = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * 4 + warp;
+  wait_prior_grid();
+  if (h >= H) return;
+  const int b = seq_of(cu, batch, i), start = cu[b];
+  const int D = dh + dr;
+  const T* qr = q + ((size_t)i * H + h) * D;
+  float m = -INFINITY, l = 0.f;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // d_v <= 256: lane's dims lane + 32u
+  for (int j = start; j <= i; ++j) {
+    float s = 0.f;
+    for (int d = lane; d < D; d += 32) {
+      const float kd = d < dh ? to_f32(kn[((size_t)j * H + h) * dh + d])
+                              : to_f32(rows[(size_t)j * ldr + r + (d - dh)]);
+      s = fmaf(to_f32(qr[d]), kd, s);
+    }
+    s = warp_sum(s) * c2;
+    const float mn = fmaxf(m, s);
+    const float alpha = ex2(m - mn), p = ex2(s - mn);
+    l = l * alpha + p;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int d = lane + 32 * u;
+      const float vd = d < dv ? to_f32(v[((size_t)j * H + h) * dv + d]) : 0.f;
+      acc[u] = fmaf(p, vd, acc[u] * alpha);
+    }
+    m = mn;
+  }
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int d = lane + 32 * u;
+    if (d < dv) o[((size_t)i * H + h) * dv + d] = from_f32<T>(acc[u] / l);
+  }
+}
+
+}  // namespace
+
+bool prefill_tc_supported(const mla_config& c) {
+  return c.dtype == MLA_BF16 && c.head_dim == 128 && c.rope_dim == 64 && c.head_dim_v == 128 &&
+         c.kv_rank % 8 == 0;
+}
+
+// Workspace: Q (n, H, d_h + d_r), K_nope (n, H * d_h), V (n, H * d_v) in dtype, then the
+// expansion's partial sums.
+struct PrefillLayout {
+  size_t q, kn, v, part, total;
+};
+
+PrefillLayout prefill_layout(const mla_config& c, int n) {
+  const size_t e = c.dtype == MLA_BF16 ? 2 : 4;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  PrefillLayout L;
+  L.q = 0;
+  L.kn = up((size_t)n * c.num_heads * (c.head_dim + c.rope_dim) * e);
+  L.v = L.kn + up((size_t)n * c.num_heads * c.head_dim * e);
+  L.part = L.v + up((size_t)n * c.num_heads * c.head_dim_v * e);
+  const int rows[2] = {c.num_heads * c.head_dim, c.num_heads * c.head_dim_v};
+  L.total = L.part + up(front_part_bytes(c, c.kv_rank, n, rows, 2, false));
+  return L;
+}
+
+cudaError_t launch_prefill(const mla_config& c, const void* q_nope, const void* q_rope,
+                           const int32_t* pos, const void* rows, const void* w_uk,
+                           const void* w_uv, const int32_t* cu, int batch, int max_seqlen, int n,
+                           void* o, void* ws, uint32_t* err, cudaStream_t st) {
+  const int H = c.num_heads, dh = c.head_dim, dr = c.rope_dim, dv = c.head_dim_v,
+            r = c.kv_rank;
+  const PrefillLayout L = prefill_layout(c, n);
+  uint8_t* w8 = (uint8_t*)ws;
+  void* q = w8 + L.q;
+  void* kn = w8 + L.kn;
+  void* v = w8 + L.v;
+  const bool bf = c.dtype == MLA_BF16;
+  // the packed, rotated query
+  const size_t csm = (size_t)std::max(1, dr / 2) * 2 * sizeof(double);
+  cudaError_t e = bf ? launch_pdl(prefill_pack_kernel<__nv_bfloat16>, dim3(n), dim3(256), csm, st,
+                                  (const __nv_bfloat16*)q_nope, (const __nv_bfloat16*)q_rope, pos,
+                                  (__nv_bfloat16*)q, H, dh, dr, c.rope_base)
+                     : launch_pdl(prefill_pack_kernel<float>, dim3(n), dim3(256), csm, st,
+                                  (const float*)q_nope, (const float*)q_rope, pos, (float*)q, H,
+                                  dh, dr, c.rope_base);
+  if (e != cudaSuccess) return e;
+  // K_nope and V from c_kv (the first r values of each cache row)
+  const void* wts[2] = {w_uk, w_uv};
+  const int wrows[2] = {H * dh, H * dv};
+  void* outs[2] = {kn, v};
+  e = launch_front_linear(c, rows, n, r, r + dr, wts, wrows, outs, 2, -1, nullptr, 0.f,
+                          w8 + L.part, err, st);
+  if (e != cudaSuccess) return e;
+  const float c2 = c.softmax_scale * 1.4426950408889634f;
+  if (prefill_tc_supported(c)) {
+    CUtensorMap tq, tkn, tkr, tv;
+    if (!make_bf16_map(&tq, q, (uint64_t)H * (dh + dr), (uint64_t)n, (uint64_t)H * (dh + dr) * 2,
+                       kPfTile) ||
+        !make_bf16_map(&tkn, kn, (uint64_t)H * dh, (uint64_t)n, (uint64_t)H * dh * 2, kPfTile) ||
+        !make_bf16_map(&tkr, rows, (uint64_t)(r + dr), (uint64_t)n, (uint64_t)(r + dr) * 2,
+                       kPfTile) ||
+        !make_bf16_map(&tv, v, (uint64_t)H * dv, (uint64_t)n, (uint64_t)H * dv * 2, kPfTile))
+      return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPfSmem);
+    if (e != cudaSuccess) return e;
+    const int qtiles = (max_seqlen + kPfTile - 1) / kPfTile;
+    PrefillArgs a{cu, (__nv_bfloat16*)o, err, batch, H, qtiles, c2};
+    return launch_pdl(prefill_tc_kernel, dim3(batch * qtiles, H), dim3(128), (size_t)kPfSmem, st,
+                      tq, tkn, tkr, tv, a, r);
+  }
+  dim3 grid(n, (H + 3) / 4);
+  return bf ? launch_pdl(prefill_simt_kernel<__nv_bfloat16>, grid, dim3(128), 0, st,
+                         (const __nv_bfloat16*)q, (const __nv_bfloat16*)kn,
+                         (const __nv_bfloat16*)rows, (const __nv_bfloat16*)v, cu, batch, H, dh,
+                         dr, dv, r + dr, r, c2, (__nv_bfloat16*)o)
+            : launch_pdl(prefill_simt_kernel<float>, grid, dim3(128), 0, st, (const float*)q,
+                         (const float*)kn, (const float*)rows, (const float*)v, cu, batch, H, dh,
+                         dr, dv, r + dr, r, c2, (float*)o);
+}
+
+size_t prefill_workspace_bytes(const mla_config& c, int n) { return prefill_layout(c, n).total; }
+
+}  // namespace mla

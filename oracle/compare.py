@@ -50,11 +50,14 @@ def per_vector_scaled_error(got: np.ndarray, ref: np.ndarray) -> float:
     return float(np.max(np.abs(got - ref) / np.maximum(r, 1e-30)))
 
 
-def within(got: np.ndarray, ref: np.ndarray, dtype: str, per_vector: bool = True):
+def within(got: np.ndarray, ref: np.ndarray, dtype: str, per_vector: bool = True,
+           out_ulps: float = 0.0):
     """(ok, metric) for the workload's storage type ("f32" or "bf16").
 
     bf16: the error scaled by the rms of the whole output, the literal unscaled bound, and
     (``per_vector``) the error of every output vector scaled by its own rms, all <= 2e-2.
+    ``out_ulps``: every element's error is first reduced by that many bfloat16 ulps of the
+    expected value (the output format's own granularity; see PROMPT_OUTPUT_ULPS).
     """
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
@@ -63,6 +66,11 @@ def within(got: np.ndarray, ref: np.ndarray, dtype: str, per_vector: bool = True
     if dtype == "f32":
         e = normwise_rel_error(got, ref)
         return e <= F32_REL_TOL, e
+    if out_ulps:
+        # the part of each error within out_ulps ulps of the expected value is not counted:
+        # compare the expected value with got moved toward it by that much
+        slack = out_ulps * bf16_ulp(ref)
+        got = ref + np.sign(got - ref) * np.maximum(np.abs(got - ref) - slack, 0.0)
     e = scaled_max_error(got, ref)
     ok = e <= BF16_SCALED_TOL and max_abs_error(got, ref) <= BF16_SCALED_TOL
     if per_vector:
@@ -80,6 +88,14 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     out[nz] = 2.0 ** (np.floor(np.log2(np.maximum(x[nz], 2.0 ** -126))) - 7)
     return out
 
+
+# A bf16 prompt (prefill) output: one query token's (H, d_v) output averages few keys in its
+# first rows and many later, so its elements can reach several times the rms of the whole
+# output or of one head's vector, where half an ulp of the bf16 result alone (0.39 % of the
+# element at the top of a binade) exceeds 2e-2 of the rms. The tensor-core pipeline also holds
+# P, K and V as bf16 MMA operands, once each. One ulp of the expected element is granted for
+# those roundings together; everything beyond it must meet the 2e-2 bar.
+PROMPT_OUTPUT_ULPS = 1.0
 
 FP32_UNIT_ROUNDOFF = 2.0 ** -24
 

@@ -264,6 +264,26 @@ def naive_decode(c_kv: np.ndarray, k_rope: np.ndarray, q_nope: np.ndarray, q_rop
     return DecodeOut(o, o_lat, lse)
 
 
+def expanded_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -> np.ndarray:
+    """Causal attention over per-head keys and values already expanded from the latent.
+
+    "MLA from scratch in PyTorch", The MLAAttention module: attn = softmax(q k^T * scale) with
+    the causal mask over the T new tokens, out = attn v. Q (T, H, D), K (L, H, D) and
+    V (L, H, d_v) hold every head's query, key ([K_nope || k_rope]) and value; the T queries
+    are the last T of the L rows. Returns o (T, H, d_v). Computed in float64 on the values
+    given, so a caller that rounds Q, K or V first gets the attention of the rounded operands.
+    """
+    Q = np.asarray(Q, dtype=F64)
+    K = np.asarray(K, dtype=F64)
+    V = np.asarray(V, dtype=F64)
+    T, L = Q.shape[0], K.shape[0]
+    s = np.einsum("thd,lhd->htl", Q, K) * scale                     # (H, T, L)
+    keep = np.arange(L)[None, :] < _causal_lengths(L, T)[:, None]     # (T, L)
+    s = np.where(keep[None], s, -np.inf)
+    p = softmax(s)
+    return np.einsum("htl,lhd->thd", p, V)
+
+
 def absorb_query(q_nope: np.ndarray, w_uk: np.ndarray, dtype=F64) -> np.ndarray:
     """q_lat[h] = W_UK[h]^T q_nope[h]: "DeepSeek MLA, Built From the Paper", 3 Matrix
     absorption -- q^T (W_UK c) = (W_UK^T q)^T c, so W_UK folds into the query once.

@@ -227,6 +227,33 @@ def test_bruteforce_small(T):
     assert np.max(np.abs(b.o - bf)) < 1e-12
 
 
+def test_expanded_attention_equals_library_causal_sdpa_and_the_naive_form():
+    # a prompt (every token new): torch's causal scaled-dot-product attention, float64
+    g = np.random.default_rng([0, 90])
+    L, H, D, dv = 11, 3, 6, 5
+    Q = g.standard_normal((L, H, D))
+    K = g.standard_normal((L, H, D))
+    V = g.standard_normal((L, H, dv))
+    o = ref.expanded_attention(Q, K, V, 0.4)
+    t = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q.transpose(1, 0, 2)), torch.from_numpy(K.transpose(1, 0, 2)),
+        torch.from_numpy(V.transpose(1, 0, 2)), is_causal=True, scale=0.4)
+    assert np.max(np.abs(o - t.numpy().transpose(1, 0, 2))) < 1e-12
+    # keys and values expanded from the latent: the naive form (pinned by brute force above),
+    # for a decode step of 3 tokens and for a whole prompt
+    for L_, T in ((9, 3), (7, 7)):
+        args, scale = _tiny_inputs(L=L_, T=T, H=2, dh=4, r=6, dr=4)
+        c, kr, qn, qr, wuk, wuv = args
+        Kx = np.concatenate([np.einsum("lr,hdr->lhd", c, wuk),
+                             np.repeat(kr[:, None, :], wuk.shape[0], axis=1)], axis=-1)
+        Vx = np.einsum("lr,hdr->lhd", c, wuv)
+        Qx = np.concatenate([qn, qr], axis=-1)
+        want = ref.naive_decode(*args, scale).o
+        assert np.max(np.abs(ref.expanded_attention(Qx, Kx, Vx, scale) - want)) < 1e-12
+        # negative control: the heads' keys swapped
+        assert np.max(np.abs(ref.expanded_attention(Qx, Kx[:, ::-1], Vx, scale) - want)) > 1e-3
+
+
 def test_causal_mask_is_not_off_by_one():
     args, scale = _tiny_inputs(L=9, T=3, H=2, dh=4, r=6, dr=4)
     c, kr, qn, qr, wuk, wuv = args
@@ -456,6 +483,24 @@ def test_tolerance_negative_controls(dtype):
     shifted = ref.naive_decode(c[:, :w.kv_rank], c[:, w.kv_rank:], d.q_nope, qr, wuk, wuv,
                                w.softmax_scale)
     assert not compare.within(shifted.o[0], o, dtype)[0]
+
+
+def test_output_ulp_allowance_admits_the_formats_rounding_only():
+    g = np.random.default_rng([0, 91])
+    exp = 0.1 * g.standard_normal((4, 64))
+    exp[2, 5] = 1.0585                        # > 5x the rms, just above a power of two
+    got = ref.round_bf16(exp)                 # the exact values, rounded to bf16 once
+    ok, e = compare.within(got, exp, "bf16")
+    assert not ok and e > 2e-2                # the format alone misses the plain bar ...
+    ok, e = compare.within(got, exp, "bf16", out_ulps=compare.PROMPT_OUTPUT_ULPS)
+    assert ok, e                              # ... and meets it with one ulp granted
+    bad = got.copy()
+    bad[2, 5] += 3 * compare.bf16_ulp(np.array(1.0585))
+    assert not compare.within(bad, exp, "bf16", out_ulps=compare.PROMPT_OUTPUT_ULPS)[0]
+    bad = got + 0.03 * np.sqrt(np.mean(exp ** 2))   # a real error on every element
+    assert not compare.within(bad, exp, "bf16", out_ulps=compare.PROMPT_OUTPUT_ULPS)[0]
+    assert not compare.within(np.zeros_like(exp), exp, "bf16",
+                              out_ulps=compare.PROMPT_OUTPUT_ULPS)[0]
 
 
 def test_needle_makes_attention_peaky():
