@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill", type=int, nargs=2, default=None, metavar=("B", "S"),
                     help="time mla_prefill on B prompts of S tokens at the workload's head shape")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time a decode step over an fp8 (e4m3) latent cache of the workload")
     ap.add_argument("--front", action="store_true",
                     help="time the decode front end (mla_project) at the workload's shape")
     ap.add_argument("--context-parallel", type=int, default=0, metavar="G",
@@ -878,10 +880,112 @@ def run_prefill(args, w):
     return 0
 
 
+# ---------------------------------------------------------------------------------------
+# FP8 latent cache: the workload's cache as e4m3 codes with per-row scales. A step appends the
+# new rows (mla_append_latent_fp8) and decodes over the fp8 pool (mla_decode_fp8).
+# ---------------------------------------------------------------------------------------
+def run_fp8(args, w):
+    import numpy as np
+    import torch
+
+    import mla_inputs as mi
+    import mla_latent_kv_44_b200 as mla
+
+    rank, world, local = dist_env()
+    if world > 1:
+        if rank == 0:
+            print(json.dumps({"metric": "fp8 decode", "unavailable":
+                              "measured on one GPU; run without torchrun"}))
+        return 0
+    dev = torch.device("cuda", 0)
+    B, T, H, r, dr = w.batch, w.new_tokens, w.num_heads, w.kv_rank, w.rope_dim
+    D, bs = r + dr, 64
+    rows = mi.total_rows(w, 0).astype(np.int64)
+    cfg = mla.Config(num_heads=H, head_dim=w.head_dim, kv_rank=r, rope_dim=dr, block_size=bs,
+                     dtype=w.dtype)
+    tdt = cfg.torch_dtype
+    nblk = [-(-int(L) // bs) for L in rows]
+    first = np.concatenate([[0], np.cumsum(nblk)])
+    table = np.zeros((B, max(nblk)), dtype=np.int32)
+    for b in range(B):
+        table[b, :nblk[b]] = first[b] + np.arange(nblk[b])
+    tab = torch.from_numpy(table).to(dev)
+    pool = torch.zeros((int(first[-1]), bs, D), dtype=torch.uint8, device=dev)
+    scale = torch.zeros((int(first[-1]), bs), dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    gamma = torch.ones(r, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(99)
+    # the cache: every sequence's rows appended (seeded N(0, 1) raw rows, like the bf16 bench)
+    for b in range(B):
+        L = int(rows[b])
+        ckv = torch.randn(L, r, generator=gen, device=dev).to(tdt)
+        kr = torch.randn(L, dr, generator=gen, device=dev).to(tdt)
+        seq = torch.full((L,), b, dtype=torch.int32, device=dev)
+        pos = torch.arange(L, dtype=torch.int32, device=dev)
+        mla.append_latent_fp8(cfg, ckv, kr, gamma, seq, pos, tab, pool, scale, err)
+    n = B * T
+    ckv_new = torch.randn(n, r, generator=gen, device=dev).to(tdt)
+    kr_new = torch.randn(n, dr, generator=gen, device=dev).to(tdt)
+    seq_new = torch.arange(B, dtype=torch.int32, device=dev).repeat_interleave(T)
+    pos_new = torch.from_numpy(np.concatenate([np.arange(L - T, L) for L in rows]).astype(
+        np.int32)).to(dev)
+    q = torch.randn(n, H, D, generator=gen, device=dev).to(tdt)
+    lens = torch.from_numpy(rows.astype(np.int32)).to(dev)
+    ws = torch.empty(mla.decode_workspace_size(cfg, B, T), dtype=torch.uint8, device=dev)
+    out = torch.empty((n, H, r), device=dev)
+    lse = torch.empty((n, H), device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    def step():
+        mla.append_latent_fp8(cfg, ckv_new, kr_new, gamma, seq_new, pos_new, tab, pool, scale,
+                              err, stream)
+        mla.decode_fp8(cfg, q, pool, scale, tab, lens, T, ws, out, lse, err, stream)
+
+    props = torch.cuda.get_device_properties(dev)
+    clock = ClockSampler(str(getattr(props, "uuid", "")), 0)
+    clock.start()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+        stream.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+    stream.synchronize()
+    clock.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())}")
+    ms = e0.elapsed_time(e1) / args.steps
+    cache_bytes = int(np.sum(rows)) * T * (D + 4)
+    gbs = cache_bytes / (ms * 1e-3) / 1e9
+    hbm, _, _, src = load_peaks()
+    print(json.dumps({
+        "metric": "MLA absorbed decode over an fp8 cache: tokens/s", "value": n / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "dtype": "fp8 e4m3 cache (per-row scale), fp32 math",
+        "data": "synthetic (seeded N(0,1) raw rows)",
+        "config": {"workload": f"{args.workload}: H={H} r={r} d_r={dr} B={B} "
+                               f"S={int(rows[0])} T={T}, fp8 pool of 64-row blocks"},
+        "ms_per_step": ms, "cache_bytes_per_step": cache_bytes,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm, "peak_source": src},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clock.summary(t0, time.time(), "warm-up and timed steps"),
+    }), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     import mla_inputs as mi
 
+    if args.fp8:
+        return run_fp8(args, mi.WORKLOADS[args.workload])
     if args.prefill:
         return run_prefill(args, mi.WORKLOADS[args.workload])
     if args.front:

@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 6
+#define MLA_ABI_VERSION 7
 
 #if defined(__GNUC__)
 #define MLA_API __attribute__((visibility("default")))
@@ -301,6 +301,38 @@ MLA_API mla_status mla_prefill(const mla_config* cfg, const void* q_nope, const 
                                const void* w_uv, const int32_t* cu_seqlens, int32_t batch,
                                int32_t max_seqlen, int32_t n_tokens, void* o, void* workspace,
                                size_t workspace_bytes, uint32_t* dev_err, void* stream);
+
+/*
+ * FP8 latent cache ("MLA from scratch in PyTorch", What's not in this implementation: the
+ * latent cache can be quantised to FP8). A pool row is r + d_r e4m3 codes (one byte each,
+ * (num_blocks, block_size, r + d_r) uint8) with one float32 scale per row
+ * (row_scale: (num_blocks, block_size)); the row reads back as code_j * scale.
+ *
+ * mla_append_latent_fp8 -- mla_append_latent's row y = [RMSNorm(c_kv) * gamma ‖ RoPE(k_rope)]
+ * (fp32), stored as scale = max_j |y_j| / 448 (1 for an all-zero row) and
+ * code_j = e4m3(y_j / scale), rounded to nearest even and saturated at 448. Arguments as
+ * mla_append_latent, with the fp8 pool and its row_scale.
+ */
+MLA_API mla_status mla_append_latent_fp8(const mla_config* cfg, const void* ckv_raw,
+                                         const void* krope_raw, const float* gamma,
+                                         const int32_t* seq_idx, const int32_t* pos,
+                                         const int32_t* block_table, int32_t batch,
+                                         int32_t max_blocks, uint8_t* pool, float* row_scale,
+                                         int32_t num_blocks, int32_t n_tokens, uint32_t* dev_err,
+                                         void* stream);
+
+/*
+ * mla_decode_fp8 -- mla_decode over an fp8 pool: every row j of the attention is
+ * code_j * row_scale[j] (fp32 arithmetic). Arguments and results as mla_decode (q in the
+ * config's dtype; the same workspace size), with the fp8 pool and its row_scale. Runs on CUDA
+ * cores: the planner, an attention kernel that dequantises the rows it stages, the combine.
+ */
+MLA_API mla_status mla_decode_fp8(const mla_config* cfg, const void* q, const uint8_t* pool,
+                                  const float* row_scale, const int32_t* block_table,
+                                  int32_t max_blocks, int32_t num_blocks, const int32_t* seq_lens,
+                                  int32_t batch, int32_t q_per_seq, void* workspace,
+                                  size_t workspace_bytes, float* out_latent, float* lse,
+                                  uint32_t* dev_err, void* stream);
 
 /* Most parts mla_combine_partials merges in one call. */
 #define MLA_MAX_COMBINE_PARTS 256

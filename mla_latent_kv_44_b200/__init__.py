@@ -69,6 +69,10 @@ def _load():
                                      _c_i32, _vp, _c_i32, _c_i32, _vp, _vp, _sz, _vp, _vp, _vp,
                                      _vp, _vp, _vp]),
         "mla_combine_partials": (_c_i32, [P, _vp, _vp, _c_i32, _c_i32, _vp, _vp, _vp]),
+        "mla_append_latent_fp8": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _vp,
+                                           _vp, _c_i32, _c_i32, _vp, _vp]),
+        "mla_decode_fp8": (_c_i32, [P, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _vp, _c_i32, _c_i32,
+                                    _vp, _sz, _vp, _vp, _vp, _vp]),
         "mla_prefill_workspace_size": (_sz, [P, _c_i32]),
         "mla_prefill": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _c_i32,
                                  _vp, _vp, _sz, _vp, _vp]),
@@ -257,6 +261,29 @@ def project(cfg: Config, front: MlaFrontConfig, x, w_dq, gamma_q, w_uq, w_qr, w_
                            int(x.shape[0]), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _ptr(dev_err),
                            _stream(stream)), "mla_project")
+
+
+def append_latent_fp8(cfg: Config, ckv_raw, krope_raw, gamma, seq_idx, pos, block_table, pool,
+                      row_scale, dev_err, stream=None):
+    """mla_append_latent_fp8: new rows as e4m3 codes (uint8 pool) with per-row scales."""
+    c = cfg.c()
+    _check(lib.mla_append_latent_fp8(ctypes.byref(c), _ptr(ckv_raw), _ptr(krope_raw), _ptr(gamma),
+                                     _ptr(seq_idx), _ptr(pos), _ptr(block_table),
+                                     int(block_table.shape[0]), int(block_table.shape[1]),
+                                     _ptr(pool), _ptr(row_scale), int(pool.shape[0]),
+                                     int(ckv_raw.shape[0]), _ptr(dev_err), _stream(stream)),
+           "mla_append_latent_fp8")
+
+
+def decode_fp8(cfg: Config, q, pool, row_scale, block_table, seq_lens, q_per_seq: int, workspace,
+               out_latent, lse, dev_err, stream=None):
+    """mla_decode_fp8: mla_decode over an fp8 pool (codes times the rows' scales)."""
+    c = cfg.c()
+    _check(lib.mla_decode_fp8(ctypes.byref(c), _ptr(q), _ptr(pool), _ptr(row_scale),
+                              _ptr(block_table), int(block_table.shape[1]), int(pool.shape[0]),
+                              _ptr(seq_lens), int(seq_lens.shape[0]), q_per_seq, _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _ptr(out_latent),
+                              _ptr(lse), _ptr(dev_err), _stream(stream)), "mla_decode_fp8")
 
 
 def prefill_workspace_size(cfg: Config, n_tokens: int) -> int:

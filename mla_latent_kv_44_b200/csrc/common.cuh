@@ -81,6 +81,7 @@ struct DecodeParams {
   int32_t* bt_chunk0;
   float* part_lse;
   float* part_o;
+  const float* row_scale;  // fp8 cache: one fp32 scale per pool row (null otherwise)
   // shapes
   int32_t H, r, dr, D, bs, max_blocks, num_blocks, batch, T, BT;
   float scale;
@@ -154,6 +155,13 @@ cudaError_t launch_attend_simt(const mla_config& c, const DecodeParams& p, cudaS
 cudaError_t launch_attend_tc(const mla_config& c, const DecodeParams& p, cudaStream_t st);
 bool tc_supported(const mla_config& c);
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t st);
+// fp8 (e4m3) latent cache: rows of the pool are codes, p.row_scale their scales
+cudaError_t launch_attend_simt_fp8(const mla_config& c, const DecodeParams& p, cudaStream_t st);
+cudaError_t launch_append_fp8(const mla_config& c, const void* ckv, const void* kr,
+                              const float* gamma, const int32_t* seq, const int32_t* pos,
+                              const int32_t* table, int batch, int max_blocks, uint8_t* pool,
+                              float* row_scale, int num_blocks, int n, uint32_t* err,
+                              cudaStream_t st);
 cudaError_t launch_output(const mla_config& c, const float* lat, const void* w_uv, void* o,
                           int n, cudaStream_t st);
 bool absorb_tc_supported(const mla_config& c);

@@ -1,4 +1,5 @@
-// CUDA-core attention stage of mla_decode (any shape; fp32 or bf16 storage, fp32 math).
+// CUDA-core attention stage of mla_decode (any shape; fp32, bf16 or fp8 e4m3 rows with a
+// per-row scale; fp32 math).
 //
 // Absorbed form ("DeepSeek MLA, Built From the Paper", 3 Matrix absorption; "MLA from scratch
 // in PyTorch", Absorbing projections): each head scores the packed query [q_lat || q_rope]
@@ -8,14 +9,28 @@
 // 32 at a time in shared memory as fp32 with an odd word stride, so that lane t computing the
 // score of row t and all lanes reading one row are both bank-conflict free. Online softmax in
 // fp32 (running max m, running sum l), exact exp, fixed summation order: deterministic.
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 
 namespace mla {
 
+// an fp8 (e4m3) cache code
+struct Fp8Code {
+  uint8_t bits;
+};
+
 constexpr int kSimtHeads = 8;   // warps (heads) per CTA
 constexpr int kSimtRows = 32;   // rows per staged tile (one per lane)
 
-template <typename T, int RW>  // RW: latent columns per lane (r <= 32 * RW)
+// e4m3 code -> float (exact: every e4m3 value is a half)
+__device__ __forceinline__ float fp8_to_f32(uint32_t code) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// TQ: the query's type, TR: the rows' (Fp8Code: codes times the row's scale)
+template <typename TQ, typename TR, int RW>  // RW: latent columns per lane (r <= 32 * RW)
 __global__ void __launch_bounds__(kSimtHeads * 32)
 attend_simt_kernel(DecodeParams p) {
   const int seg_id = blockIdx.x;
@@ -36,9 +51,10 @@ attend_simt_kernel(DecodeParams p) {
   float* s_rows = smem;                          // kSimtRows x ld
   float* s_q = smem + kSimtRows * ld;            // kSimtHeads x D
   int* s_ok = (int*)(s_q + kSimtHeads * D);      // kSimtRows
+  float* s_scale = (float*)(s_ok + kSimtRows);   // kSimtRows (fp8 rows)
 
-  const T* Q = (const T*)p.q;
-  const T* pool = (const T*)p.pool;
+  const TQ* Q = (const TQ*)p.q;
+  const TR* pool = (const TR*)p.pool;
   for (int idx = threadIdx.x; idx < kSimtHeads * D; idx += blockDim.x) {
     const int hh = blockIdx.y * kSimtHeads + idx / D;
     s_q[idx] = hh < p.H ? to_f32(Q[((size_t)bt * p.H + hh) * D + idx % D]) : 0.f;
@@ -61,6 +77,8 @@ attend_simt_kernel(DecodeParams p) {
         else set_error(p.err, MLA_DEV_OOB_BLOCK);
       }
       s_ok[threadIdx.x] = ok;
+      if (sizeof(TR) == 1)
+        s_scale[threadIdx.x] = ok ? p.row_scale[(size_t)(ok - 1) * p.bs + tok % p.bs] : 0.f;
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < kSimtRows * quads; idx += blockDim.x) {
@@ -69,10 +87,17 @@ attend_simt_kernel(DecodeParams p) {
       float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
       if (ok) {
         const int tok = t0 + t;
-        const T* row = pool + ((size_t)(ok - 1) * p.bs + tok % p.bs) * D + 4 * qd;
-        if (sizeof(T) == 4) {
+        const TR* row = pool + ((size_t)(ok - 1) * p.bs + tok % p.bs) * D + 4 * qd;
+        if (sizeof(TR) == 4) {
           const float4 v = *(const float4*)row;
           v0 = v.x; v1 = v.y; v2 = v.z; v3 = v.w;
+        } else if (sizeof(TR) == 1) {
+          const uint32_t u = *(const uint32_t*)row;
+          const float sc = s_scale[t];
+          v0 = fp8_to_f32(u & 0xffu) * sc;
+          v1 = fp8_to_f32((u >> 8) & 0xffu) * sc;
+          v2 = fp8_to_f32((u >> 16) & 0xffu) * sc;
+          v3 = fp8_to_f32(u >> 24) * sc;
         } else {
           const uint2 u = *(const uint2*)row;
           const __nv_bfloat162 a = *(const __nv_bfloat162*)&u.x;
@@ -132,28 +157,34 @@ attend_simt_kernel(DecodeParams p) {
   }
 }
 
-template <typename T, int RW>
+template <typename TQ, typename TR, int RW>
 static cudaError_t simt_go(const DecodeParams& p, cudaStream_t st) {
   const size_t smem = sizeof(float) * (kSimtRows * (p.D + 1) + kSimtHeads * p.D) +
-                      sizeof(int) * kSimtRows;
-  auto k = attend_simt_kernel<T, RW>;
+                      (sizeof(int) + sizeof(float)) * kSimtRows;
+  auto k = attend_simt_kernel<TQ, TR, RW>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(kRanges + p.BT, (p.H + kSimtHeads - 1) / kSimtHeads);
   return launch_pdl(k, grid, dim3(kSimtHeads * 32), smem, st, p);
 }
 
-template <typename T>
+template <typename TQ, typename TR>
 static cudaError_t simt_dispatch(const DecodeParams& p, cudaStream_t st) {
-  if (p.r <= 64) return simt_go<T, 2>(p, st);
-  if (p.r <= 128) return simt_go<T, 4>(p, st);
-  if (p.r <= 256) return simt_go<T, 8>(p, st);
-  if (p.r <= 512) return simt_go<T, 16>(p, st);
-  return simt_go<T, 32>(p, st);
+  if (p.r <= 64) return simt_go<TQ, TR, 2>(p, st);
+  if (p.r <= 128) return simt_go<TQ, TR, 4>(p, st);
+  if (p.r <= 256) return simt_go<TQ, TR, 8>(p, st);
+  if (p.r <= 512) return simt_go<TQ, TR, 16>(p, st);
+  return simt_go<TQ, TR, 32>(p, st);
 }
 
 cudaError_t launch_attend_simt(const mla_config& c, const DecodeParams& p, cudaStream_t st) {
-  return c.dtype == MLA_BF16 ? simt_dispatch<__nv_bfloat16>(p, st) : simt_dispatch<float>(p, st);
+  return c.dtype == MLA_BF16 ? simt_dispatch<__nv_bfloat16, __nv_bfloat16>(p, st)
+                             : simt_dispatch<float, float>(p, st);
+}
+
+cudaError_t launch_attend_simt_fp8(const mla_config& c, const DecodeParams& p, cudaStream_t st) {
+  return c.dtype == MLA_BF16 ? simt_dispatch<__nv_bfloat16, Fp8Code>(p, st)
+                             : simt_dispatch<float, Fp8Code>(p, st);
 }
 
 }  // namespace mla

@@ -76,6 +76,7 @@ DecodeParams make_params(const mla_config* cfg, const void* q, const void* pool,
   p.bt_chunk0 = reinterpret_cast<int32_t*>(ws + L.bt_chunk0);
   p.part_lse = reinterpret_cast<float*>(ws + L.part_lse);
   p.part_o = reinterpret_cast<float*>(ws + L.part_o);
+  p.row_scale = nullptr;
   p.H = cfg->num_heads;
   p.r = cfg->kv_rank;
   p.dr = cfg->rope_dim;
@@ -334,6 +335,52 @@ mla_status mla_decode_stages(const mla_config* cfg, int32_t stages, const void* 
   if (e == cudaSuccess && (stages & MLA_STAGE_ATTEND))
     e = use_tc ? launch_attend_tc(*cfg, p, st) : launch_attend_simt(*cfg, p, st);
   if (e == cudaSuccess && (stages & MLA_STAGE_COMBINE)) e = launch_combine(p, st);
+  return from_cuda(e);
+}
+
+mla_status mla_append_latent_fp8(const mla_config* cfg, const void* ckv_raw,
+                                 const void* krope_raw, const float* gamma,
+                                 const int32_t* seq_idx, const int32_t* pos,
+                                 const int32_t* block_table, int32_t batch, int32_t max_blocks,
+                                 uint8_t* pool, float* row_scale, int32_t num_blocks,
+                                 int32_t n_tokens, uint32_t* dev_err, void* stream) {
+  if (!valid_config(cfg) || n_tokens < 0 || batch < 0) return MLA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return MLA_OK;
+  if (!ckv_raw || (cfg->rope_dim > 0 && !krope_raw) || !gamma || !seq_idx || !pos ||
+      !block_table || !pool || !row_scale || !dev_err)
+    return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || max_blocks < 1 || num_blocks < 1) return MLA_ERR_INVALID_ARG;
+  if (n_tokens > (1 << 26)) return MLA_ERR_UNSUPPORTED;
+  return from_cuda(launch_append_fp8(*cfg, ckv_raw, krope_raw, gamma, seq_idx, pos, block_table,
+                                     batch, max_blocks, pool, row_scale, num_blocks, n_tokens,
+                                     dev_err, (cudaStream_t)stream));
+}
+
+mla_status mla_decode_fp8(const mla_config* cfg, const void* q, const uint8_t* pool,
+                          const float* row_scale, const int32_t* block_table, int32_t max_blocks,
+                          int32_t num_blocks, const int32_t* seq_lens, int32_t batch,
+                          int32_t q_per_seq, void* workspace, size_t workspace_bytes,
+                          float* out_latent, float* lse, uint32_t* dev_err, void* stream) {
+  if (!valid_config(cfg) || batch < 0 || q_per_seq < 1) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  if (!q || !pool || !row_scale || !block_table || !seq_lens || !workspace || !out_latent ||
+      !dev_err)
+    return MLA_ERR_INVALID_ARG;
+  if (max_blocks < 1 || num_blocks < 1) return MLA_ERR_INVALID_ARG;
+  const int64_t bt = (int64_t)batch * q_per_seq;
+  if (bt > (1 << 24)) return MLA_ERR_UNSUPPORTED;
+  const size_t need = mla_decode_workspace_size(cfg, batch, q_per_seq);
+  if (need == 0) return MLA_ERR_INVALID_ARG;
+  if (workspace_bytes < need || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+  if (!aligned(pool, 16) || !aligned(q, 16) || !aligned(out_latent, 16))
+    return MLA_ERR_INVALID_ARG;
+  DecodeParams p = make_params(cfg, q, pool, block_table, max_blocks, num_blocks, seq_lens, batch,
+                               q_per_seq, workspace, out_latent, lse, dev_err);
+  p.row_scale = row_scale;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = launch_plan(p, st);
+  if (e == cudaSuccess) e = launch_attend_simt_fp8(*cfg, p, st);
+  if (e == cudaSuccess) e = launch_combine(p, st);
   return from_cuda(e);
 }
 

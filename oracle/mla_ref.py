@@ -103,6 +103,32 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
     return out
 
 
+def round_fp8_e4m3(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest FP8 E4M3 value, ties to even, saturating at +-448.
+
+    E4M3 ("MLA from scratch in PyTorch", What's not in this implementation: the latent cache
+    can be quantised to FP8): a sign, 4 exponent bits with bias 7 and 3 mantissa bits, so the
+    values in [2^e, 2^(e+1)) are spaced 2^(e-3) for e >= -6, and below 2^-6 the subnormals are
+    spaced 2^-9; the largest finite value is 1.75 * 2^8 = 448.
+    """
+    x = np.asarray(x, dtype=F64)
+    a = np.abs(x)
+    e = np.maximum(np.floor(np.log2(np.maximum(a, 2.0 ** -30))), -6.0)
+    step = 2.0 ** (e - 3.0)
+    y = np.minimum(np.round(a / step) * step, 448.0)   # np.round: half to even
+    return np.copysign(y, x)
+
+
+def quantize_rows_fp8(rows: np.ndarray):
+    """(codes, scale) of cache rows stored as E4M3 with one scale per row: scale =
+    max |row| / 448 (1 for an all-zero row), codes = E4M3(row / scale); a row reads back as
+    codes * scale. rows (..., D) -> codes (..., D) as float values, scale (...,)."""
+    rows = np.asarray(rows, dtype=F64)
+    amax = np.max(np.abs(rows), axis=-1)
+    scale = np.where(amax > 0, amax / 448.0, 1.0)
+    return round_fp8_e4m3(rows / scale[..., None]), scale
+
+
 def softmax(s: np.ndarray, axis: int = -1) -> np.ndarray:
     """exp(s - max) / sum(exp(s - max)); entries equal to -inf get exactly 0."""
     m = np.max(s, axis=axis, keepdims=True)

@@ -397,6 +397,29 @@ def test_round_bf16_matches_library_conversion():
     assert ref.round_bf16(np.array([1 + 3 * 2 ** -8]))[0] == 1 + 2 ** -6
 
 
+def test_round_fp8_e4m3_matches_library_conversion():
+    # every E4M3 value, the midpoints between neighbours (ties to even), points just off the
+    # midpoints, subnormals, and random values; torch's float8_e4m3fn conversion bit for bit
+    codes = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    vals = np.unique(codes[np.isfinite(codes)])
+    mids = (vals[1:] + vals[:-1]) / 2
+    g = np.random.default_rng([0, 92])
+    x = np.concatenate([vals, mids, mids * (1 + 2.0 ** -20), mids * (1 - 2.0 ** -20),
+                        g.uniform(-448, 448, 2000), g.uniform(-0.02, 0.02, 500),
+                        [0.0, -0.0, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -11, 447.9, -447.9]])
+    x = x.astype(np.float32)   # the library converts from float32
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).float().numpy()
+    got = ref.round_fp8_e4m3(x.astype(np.float64))
+    assert np.array_equal(got.astype(np.float32), want)
+    # the grid: 1 + k/8 between 1 and 2, spacing 2^-9 among the subnormals, 448 the largest
+    assert ref.round_fp8_e4m3(np.array([1.0 + 1 / 16]))[0] == 1.0      # tie -> even mantissa
+    assert ref.round_fp8_e4m3(np.array([1.0 + 3 / 16]))[0] == 1.25
+    assert ref.round_fp8_e4m3(np.array([1000.0]))[0] == 448.0          # saturation
+    codes_, scale = ref.quantize_rows_fp8(np.array([[0.5, -2.0, 1.0], [0.0, 0.0, 0.0]]))
+    assert scale[0] == 2.0 / 448 and scale[1] == 1.0
+    assert np.array_equal(codes_[0], [112.0, -448.0, 224.0]) and not codes_[1].any()
+
+
 def test_project_layer_matches_library_linear():
     w = mi.WORKLOADS["small_fp32"]
     d = mi.layer_draw(mi.scaled(w, batch=2, cached=5))
