@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 7
+#define MLA_ABI_VERSION 8
 
 #if defined(__GNUC__)
 #define MLA_API __attribute__((visibility("default")))
@@ -321,11 +321,18 @@ MLA_API mla_status mla_append_latent_fp8(const mla_config* cfg, const void* ckv_
                                          int32_t num_blocks, int32_t n_tokens, uint32_t* dev_err,
                                          void* stream);
 
+/* Workspace of mla_decode_fp8 in bytes (0 for an invalid configuration); 256-byte aligned. */
+MLA_API size_t mla_decode_fp8_workspace_size(const mla_config* cfg, int32_t batch,
+                                             int32_t q_per_seq, int32_t max_blocks);
+
 /*
  * mla_decode_fp8 -- mla_decode over an fp8 pool: every row j of the attention is
- * code_j * row_scale[j] (fp32 arithmetic). Arguments and results as mla_decode (q in the
- * config's dtype; the same workspace size), with the fp8 pool and its row_scale. Runs on CUDA
- * cores: the planner, an attention kernel that dequantises the rows it stages, the combine.
+ * code_j * row_scale[j]. Arguments and results as mla_decode (q in the config's dtype), with
+ * the fp8 pool, its row_scale and a workspace of mla_decode_fp8_workspace_size bytes. Where
+ * mla_decode would take the tensor-core attention (bf16, its shape), the step's blocks are
+ * first expanded to bf16 in the workspace (batch x max_blocks blocks of scratch, rounded to
+ * nearest even) and that kernel runs over them; otherwise the CUDA-core attention reads the
+ * codes directly (fp32 arithmetic).
  */
 MLA_API mla_status mla_decode_fp8(const mla_config* cfg, const void* q, const uint8_t* pool,
                                   const float* row_scale, const int32_t* block_table,

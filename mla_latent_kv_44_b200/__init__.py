@@ -71,6 +71,7 @@ def _load():
         "mla_combine_partials": (_c_i32, [P, _vp, _vp, _c_i32, _c_i32, _vp, _vp, _vp]),
         "mla_append_latent_fp8": (_c_i32, [P, _vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _vp,
                                            _vp, _c_i32, _c_i32, _vp, _vp]),
+        "mla_decode_fp8_workspace_size": (_sz, [P, _c_i32, _c_i32, _c_i32]),
         "mla_decode_fp8": (_c_i32, [P, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _vp, _c_i32, _c_i32,
                                     _vp, _sz, _vp, _vp, _vp, _vp]),
         "mla_prefill_workspace_size": (_sz, [P, _c_i32]),
@@ -273,6 +274,11 @@ def append_latent_fp8(cfg: Config, ckv_raw, krope_raw, gamma, seq_idx, pos, bloc
                                      _ptr(pool), _ptr(row_scale), int(pool.shape[0]),
                                      int(ckv_raw.shape[0]), _ptr(dev_err), _stream(stream)),
            "mla_append_latent_fp8")
+
+
+def decode_fp8_workspace_size(cfg: Config, batch: int, q_per_seq: int, max_blocks: int) -> int:
+    return int(lib.mla_decode_fp8_workspace_size(ctypes.byref(cfg.c()), batch, q_per_seq,
+                                                 max_blocks))
 
 
 def decode_fp8(cfg: Config, q, pool, row_scale, block_table, seq_lens, q_per_seq: int, workspace,

@@ -20,6 +20,11 @@ cudaError_t launch_front_linear(const mla_config& c, const void* x, int n, int K
                                 const void* const* w, const int* rows, void* const* out, int nseg,
                                 int norm_seg, const float* gamma, float eps, void* part,
                                 uint32_t* err, cudaStream_t st);
+// fp8_cache.cu: the step's fp8 blocks expanded to bf16 for the tensor-core decode
+cudaError_t launch_dequant_fp8(const uint8_t* pool, const float* row_scale, const int32_t* table,
+                               const int32_t* seq_lens, int batch, int max_blocks, int num_blocks,
+                               int bs, int D, void* out, int32_t* out_table, uint32_t* err,
+                               cudaStream_t st);
 // prefill_tc.cu: mla_prefill
 bool prefill_tc_supported(const mla_config& c);
 size_t prefill_workspace_bytes(const mla_config& c, int n);
@@ -356,6 +361,31 @@ mla_status mla_append_latent_fp8(const mla_config* cfg, const void* ckv_raw,
                                      dev_err, (cudaStream_t)stream));
 }
 
+// The fp8 decode's workspace: mla_decode's, then (tensor-core path) the scratch block table
+// (batch x max_blocks int32) and the scratch bf16 pool (batch x max_blocks blocks).
+struct Fp8Layout {
+  size_t table, pool, total;
+  bool tc;
+};
+
+Fp8Layout fp8_layout(const mla_config& c, int batch, int q_per_seq, int max_blocks) {
+  Fp8Layout L{};
+  const size_t dec = mla_decode_workspace_size(&c, batch, q_per_seq);
+  L.tc = c.decode_kernel != MLA_DECODE_SIMT && tc_supported(c);
+  L.table = (dec + 255) / 256 * 256;
+  L.pool = L.table + ((size_t)batch * max_blocks * 4 + 255) / 256 * 256;
+  L.total = L.tc ? L.pool + (size_t)batch * max_blocks * c.block_size *
+                                (c.kv_rank + c.rope_dim) * 2
+                 : dec;
+  return L;
+}
+
+size_t mla_decode_fp8_workspace_size(const mla_config* cfg, int32_t batch, int32_t q_per_seq,
+                                     int32_t max_blocks) {
+  if (mla_decode_workspace_size(cfg, batch, q_per_seq) == 0 || max_blocks < 1) return 0;
+  return fp8_layout(*cfg, batch, q_per_seq, max_blocks).total;
+}
+
 mla_status mla_decode_fp8(const mla_config* cfg, const void* q, const uint8_t* pool,
                           const float* row_scale, const int32_t* block_table, int32_t max_blocks,
                           int32_t num_blocks, const int32_t* seq_lens, int32_t batch,
@@ -369,16 +399,34 @@ mla_status mla_decode_fp8(const mla_config* cfg, const void* q, const uint8_t* p
   if (max_blocks < 1 || num_blocks < 1) return MLA_ERR_INVALID_ARG;
   const int64_t bt = (int64_t)batch * q_per_seq;
   if (bt > (1 << 24)) return MLA_ERR_UNSUPPORTED;
-  const size_t need = mla_decode_workspace_size(cfg, batch, q_per_seq);
-  if (need == 0) return MLA_ERR_INVALID_ARG;
-  if (workspace_bytes < need || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+  if (mla_decode_workspace_size(cfg, batch, q_per_seq) == 0) return MLA_ERR_INVALID_ARG;
+  const Fp8Layout L = fp8_layout(*cfg, batch, q_per_seq, max_blocks);
+  if (workspace_bytes < L.total || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
   if (!aligned(pool, 16) || !aligned(q, 16) || !aligned(out_latent, 16))
     return MLA_ERR_INVALID_ARG;
+  if ((int64_t)batch * max_blocks > (1 << 24)) return MLA_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (L.tc) {
+    // the step's blocks in bf16, then the tensor-core decode over them
+    uint8_t* ws = (uint8_t*)workspace;
+    int32_t* table_s = (int32_t*)(ws + L.table);
+    void* pool_s = ws + L.pool;
+    e = launch_dequant_fp8(pool, row_scale, block_table, seq_lens, batch, max_blocks, num_blocks,
+                           cfg->block_size, cfg->kv_rank + cfg->rope_dim, pool_s, table_s,
+                           dev_err, st);
+    const DecodeParams p = make_params(cfg, q, pool_s, table_s, max_blocks, batch * max_blocks,
+                                       seq_lens, batch, q_per_seq, workspace, out_latent, lse,
+                                       dev_err);
+    if (e == cudaSuccess) e = launch_plan(p, st);
+    if (e == cudaSuccess) e = launch_attend_tc(*cfg, p, st);
+    if (e == cudaSuccess) e = launch_combine(p, st);
+    return from_cuda(e);
+  }
   DecodeParams p = make_params(cfg, q, pool, block_table, max_blocks, num_blocks, seq_lens, batch,
                                q_per_seq, workspace, out_latent, lse, dev_err);
   p.row_scale = row_scale;
-  cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = launch_plan(p, st);
+  e = launch_plan(p, st);
   if (e == cudaSuccess) e = launch_attend_simt_fp8(*cfg, p, st);
   if (e == cudaSuccess) e = launch_combine(p, st);
   return from_cuda(e);

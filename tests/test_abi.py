@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(mla):
 
 
 def test_abi_version_and_status_strings(mla):
-    assert mla.abi_version() == 7
+    assert mla.abi_version() == 8
     assert mla.status_string(0) == "MLA_OK"
     assert mla.status_string(4) == "MLA_ERR_WORKSPACE"
     assert mla.status_string(99) == "MLA_ERR_UNKNOWN"

@@ -6,8 +6,9 @@ rounding pinned to torch's float8_e4m3fn). The device computes the row in fp32, 
 come out as the other neighbour only where row / scale lies within the fp32 arithmetic's
 relative error (1e-5 here, from r-term sums of squares) of a rounding midpoint; every other
 code must be equal, bit for bit. The decode over the fp8 pool is compared with the oracle's
-attention over its own dequantised rows (codes * scale), within the bar of the 8-bit storage
-type's nearest one (2e-2, as bf16). CPU: argument validation.
+attention over its own dequantised rows (codes * scale; rounded to bf16 where the tensor-core
+path consumes them as bf16 operands), within the bar of the 8-bit storage type's nearest one
+(2e-2, as bf16). CPU: argument validation.
 """
 import ctypes
 
@@ -46,7 +47,9 @@ def test_fp8_calls_validate_arguments(mla):
         assert app(ctypes.byref(c), *a, 2, 4, 256, 256, 8, 4, 256, None) == mla.MLA_ERR_INVALID_ARG
     assert app(ctypes.byref(c), *args, 2, 4, 256, None, 8, 4, 256, None) == mla.MLA_ERR_INVALID_ARG
     dec = mla.lib.mla_decode_fp8
-    ws = mla.lib.mla_decode_workspace_size(ctypes.byref(c), 2, 1)
+    ws = mla.lib.mla_decode_fp8_workspace_size(ctypes.byref(c), 2, 1, 4)
+    # the tensor-core path's scratch: 2 sequences x 4 blocks of bf16 rows
+    assert ws >= mla.lib.mla_decode_workspace_size(ctypes.byref(c), 2, 1) + 8 * 64 * 576 * 2
     call = lambda scale, wsz, wsp=256, pool=256: dec(  # noqa: E731
         ctypes.byref(c), 256, pool, scale, 256, 4, 8, 256, 2, 1, wsp, wsz, 256, None, 256, None)
     assert call(None, ws) == mla.MLA_ERR_INVALID_ARG
@@ -127,6 +130,10 @@ def test_decode_fp8_matches_the_oracle(mla, name, lens, T):
                                                                          bs=bs)
     H, r = w.num_heads, w.kv_rank
     wuk, _ = (mi.storage_round(w, x) for x in mi.up_projection_weights(w, 7))
+    # where the tensor-core attention runs (bf16, H = 128, r = 512, d_r = 64, 64-row blocks),
+    # the rows are expanded to bf16 operands first, as a bf16 cache's rows are bf16 on both
+    # sides; the CUDA-core path reads codes * scale in fp32
+    tc = (w.dtype == "bf16" and H == 128 and r == 512 and w.rope_dim == 64 and bs == 64)
     Qs, exp = [], []
     for b, L in enumerate(lens):
         c1, k1, qn, qr = draws[b]
@@ -134,12 +141,14 @@ def test_decode_fp8_matches_the_oracle(mla, name, lens, T):
         Qb = mi.storage_round(w, Q)
         Qs.append(Qb)
         deq = codes[b] * scales[b][:, None]
+        if tc:
+            deq = ref.round_bf16(deq)
         exp.append(ref.latent_attention(Qb, deq, r, w.softmax_scale, T))
     tdt = cfg.torch_dtype
     q = torch.from_numpy(np.ascontiguousarray(np.concatenate(Qs), np.float32)).cuda().to(tdt)
     lens_t = torch.tensor(lens, dtype=torch.int32).cuda()
-    ws = torch.empty(mla.decode_workspace_size(cfg, len(lens), T), dtype=torch.uint8,
-                     device="cuda")
+    ws = torch.empty(mla.decode_fp8_workspace_size(cfg, len(lens), T, table.shape[1]),
+                     dtype=torch.uint8, device="cuda")
     out = torch.empty((len(lens) * T, H, r), device="cuda")
     lse = torch.empty((len(lens) * T, H), device="cuda")
     mla.decode_fp8(cfg, q, pool, scale, tab, lens_t, T, ws, out, lse, err)
