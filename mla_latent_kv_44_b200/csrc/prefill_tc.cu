@@ -9,14 +9,17 @@
 // r + d_r = 576), so K and V are expanded once per key: one split-K weight-stream launch of the
 // front end's kernel (W_UK and W_UV as two segments, c_kv read in place from the cache rows).
 // A pack kernel writes the query as [q_nope ‖ RoPE(q_rope)] (angles in double).
-// The attention kernel takes one CTA per (128-query tile, head) of a sequence (DeepSeek-V2's
-// head shape: d_h = 128, d_r = 64, d_v = 128, bf16): the query tile stays in shared memory;
-// per 128-key tile, TMA brings the key tile (K_nope of the head and the shared k_rope: three
-// 64-wide slabs) and the value tile, one thread issues S = Q K^T (M = 128 queries, N = 128
-// keys, 12 K-steps) into TMEM, the four warps (a thread per query row) take the row maximum,
-// rescale O in TMEM when the maximum grows by more than 2^8 (exp2 units), write P in bf16 into
-// shared memory as the A operand, and one thread issues O += P V (N = 128, V MN-major). Tiles
-// above the diagonal are skipped; the diagonal tile is masked. Other shapes and fp32 take a
+// The attention kernel takes one CTA per (two adjacent 128-query tiles A and B, head) of a
+// sequence (DeepSeek-V2's head shape: d_h = 128, d_r = 64, d_v = 128, bf16). Both query tiles
+// stay in shared memory and share every key and value tile TMA brings (K_nope of the head and
+// the shared k_rope: three 64-wide slabs; V: two). One thread issues S_A = Q_A K^T and
+// S_B = Q_B K^T (M = 128 queries, N = 128 keys, 12 K-steps) into their TMEM columns, and
+// O_x += P_x V as each tile's P is ready (N = 128, V MN-major, P read from TMEM: the TS form).
+// Two groups of four warps take a tile each (a thread per query row): row maximum, rescale of
+// O in TMEM when the maximum grows by more than 2^8 (exp2 units), P in bf16 written back over
+// the tile's S columns. While one group's softmax runs the tensor core works on the other
+// tile, so the two alternate. Key tiles above a query tile's diagonal are skipped; the
+// diagonal tile is masked. Other shapes and fp32 take a
 // CUDA-core kernel (a warp per (query, head), online softmax over the keys).
 // Every mbarrier wait gives up after 1 s: the kernel then sets MLA_DEV_WAIT_TIMEOUT, waits
 // (bounded) for what it issued, frees TMEM and returns.
@@ -38,15 +41,17 @@ cudaError_t launch_front_linear(const mla_config& c, const void* x, int n, int K
 namespace {
 
 constexpr unsigned long long kPfTimeoutNs = 1000000000ull;
-constexpr int kPfTile = 128;                   // queries per CTA = keys per tile
+constexpr int kPfTile = 128;                   // queries per tile = keys per tile
 constexpr int kPfSlabBytes = kPfTile * 128;    // 128 rows x 64 bf16: 16 KB
-constexpr int kPfQ = 0;                        // query: 3 slabs (q_nope 0-63, 64-127, q_rope)
-constexpr int kPfK = kPfQ + 3 * kPfSlabBytes;  // keys: 3 slabs (K_nope 0-63, 64-127, k_rope)
+constexpr int kPfQ = 0;                        // two query tiles: 3 slabs each (q_nope 0-63,
+                                               // 64-127, q_rope)
+constexpr int kPfK = kPfQ + 6 * kPfSlabBytes;  // keys: 3 slabs (K_nope 0-63, 64-127, k_rope)
 constexpr int kPfV = kPfK + 3 * kPfSlabBytes;  // values: 2 slabs (d_v 0-63, 64-127), MN-major
-constexpr int kPfP = kPfV + 2 * kPfSlabBytes;  // P: 2 slabs (keys 0-63, 64-127), K-major
-constexpr int kPfBar = kPfP + 2 * kPfSlabBytes;
-constexpr int kPfSmem = kPfBar + 64 + 1024;
-constexpr uint32_t kPfTmemCols = 256;          // S: columns 0-127, O: 128-255
+constexpr int kPfBar = kPfV + 2 * kPfSlabBytes;
+constexpr int kPfSmem = kPfBar + 128 + 1024;
+constexpr int kPfThreads = 320;                // warps 0-3, 4-7: softmax of tiles A, B;
+                                               // 8: TMA; 9: MMA issue
+constexpr uint32_t kPfTmemCols = 512;          // S_A, S_B, O_A, O_B: 128 columns each
 
 __device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
   if (mbar_try(bar, parity)) return true;
@@ -58,6 +63,22 @@ __device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, uint32_t*
     }
   }
   return true;
+}
+
+// Warp-wide bounded wait: the same result in every lane.
+__device__ __forceinline__ bool warp_all_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
+  bool done = false, ok = true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    done = __all_sync(0xffffffffu, mbar_try(bar, parity));
+    if (done) break;
+    if (__any_sync(0xffffffffu, globaltimer() - t0 > kPfTimeoutNs)) {
+      if ((threadIdx.x & 31) == 0) set_error(err, MLA_DEV_WAIT_TIMEOUT);
+      ok = false;
+      break;
+    }
+  }
+  return ok;
 }
 
 // The sequence of token index i: cu_seqlens[b] <= i < cu_seqlens[b + 1] (binary search).
@@ -111,13 +132,13 @@ struct PrefillArgs {
   const int32_t* cu;
   __nv_bfloat16* o;
   uint32_t* err;
-  int batch, H, qtiles;  // qtiles: query tiles per sequence in the grid (max_seqlen / 128)
-  float c2;              // softmax scale * log2(e)
+  int batch, H, pairs;  // pairs: query-tile pairs per sequence in the grid (max_seqlen / 256)
+  float c2;             // softmax scale * log2(e)
 };
 
-// Grid (batch * qtiles, H); 128 threads. TMA maps: q (n, H * 192), kn (n, H * 128),
+// Grid (batch * pairs, H); 320 threads. TMA maps: q (n, H * 192), kn (n, H * 128),
 // rows (n, r + 64): k_rope at column r, v (n, H * 128); all with 128-row boxes of 64 columns.
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kPfThreads)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kn,
                   const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_v,
                   const PrefillArgs a, int r) {
@@ -125,12 +146,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sb = saddr(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.x / a.qtiles, qt = blockIdx.x - b * a.qtiles, h = blockIdx.y;
+  const int b = blockIdx.x / a.pairs, pr = blockIdx.x - b * a.pairs, h = blockIdx.y;
+  // barriers: q, k, v, kfree, vfree, s[2], p[2], o[2], final
   const uint32_t bar_q = sb + kPfBar, bar_k = bar_q + 8, bar_v = bar_q + 16;
-  const uint32_t bar_s = bar_q + 24, bar_o = bar_q + 32;
-  uint32_t* tmem_slot = (uint32_t*)(smem + kPfBar + 40);
+  const uint32_t bar_kfree = bar_q + 24, bar_vfree = bar_q + 32;
+  const uint32_t bar_s = bar_q + 40, bar_p = bar_q + 56, bar_o = bar_q + 72;
+  const uint32_t bar_fin = bar_q + 88;
+  uint32_t* tmem_slot = (uint32_t*)(smem + kPfBar + 96);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 5; ++i) mbar_init(bar_q + 8 * i, 1);
+    for (int i = 0; i < 12; ++i) mbar_init(bar_q + 8 * i, (i == 7 || i == 8) ? 4 : 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -146,182 +170,196 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t tmem = *tmem_slot;
   wait_prior_grid();
   const int start = a.cu[b], len = a.cu[b + 1] - start;
-  const int q0 = qt * kPfTile;
+  const int q0 = pr * 2 * kPfTile;
+  // key tiles of each query tile: 0 .. its diagonal (none when the tile starts past the end)
+  int nkt[2];
+  for (int g = 0; g < 2; ++g) {
+    const int qg = q0 + g * kPfTile;
+    nkt[g] = qg < len ? (min(len, qg + kPfTile) - 1) / kPfTile + 1 : 0;
+  }
+  const int nk = max(nkt[0], nkt[1]);  // tile B's count when it has rows
   bool ok = true;
-  int issued_k = 0, issued_v = 0, done_s = 0, done_o = 0;  // phases, for the abort drain
-  if (q0 < len) {
-    const int nkt = (min(len, q0 + kPfTile) - 1) / kPfTile + 1;  // key tiles 0 .. diagonal
-    auto load_k = [&](int j) {
-      mbar_expect_tx(bar_k, 3 * kPfSlabBytes);
-      for (int s = 0; s < 2; ++s)
-        tma_load(sb + kPfK + s * kPfSlabBytes, &tm_kn, bar_k, h * 128 + 64 * s,
-                 start + j * kPfTile);
-      tma_load(sb + kPfK + 2 * kPfSlabBytes, &tm_kr, bar_k, r, start + j * kPfTile);
-    };
-    auto load_v = [&](int j) {
-      mbar_expect_tx(bar_v, 2 * kPfSlabBytes);
-      for (int s = 0; s < 2; ++s)
-        tma_load(sb + kPfV + s * kPfSlabBytes, &tm_v, bar_v, h * 128 + 64 * s,
-                 start + j * kPfTile);
-    };
-    if (threadIdx.x == 0) {
-      mbar_expect_tx(bar_q, 3 * kPfSlabBytes);
-      for (int s = 0; s < 3; ++s)
-        tma_load(sb + kPfQ + s * kPfSlabBytes, &tm_q, bar_q, h * 192 + 64 * s, start + q0);
-      load_k(0);
-      load_v(0);
-    }
-    issued_k = issued_v = 1;
-    const int qi = q0 + threadIdx.x;  // this thread's query (TMEM lane threadIdx.x)
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    const uint32_t t_s = tmem + lane_base, t_o = tmem + lane_base + 128;
-    float m_ref = 0.f, l = 0.f;
-    if (threadIdx.x == 0) ok = pf_wait(bar_q, 0, a.err);
-    ok = __syncthreads_and(ok);
-    for (int j = 0; j < nkt && ok; ++j) {
-      // S = Q K_j^T
-      if (threadIdx.x == 0) {
-        ok = pf_wait(bar_k, j & 1, a.err);
-        if (ok) {
-          tc_after();
-          const uint32_t id = idesc(128, 128, 0, 0);
-          for (int ks = 0; ks < 12; ++ks) {
-            const uint32_t off = (uint32_t)(ks >> 2) * kPfSlabBytes + 32u * (uint32_t)(ks & 3);
-            mma_ss(tmem, sdesc(sb + kPfQ + off, 16, 1024, 2), sdesc(sb + kPfK + off, 16, 1024, 2),
-                   id, ks > 0 ? 1u : 0u);
-          }
-          tc_commit(bar_s);
+  if (nkt[0] > 0) {
+    if (warp == 8) {
+      // ---------------------------------------------------------------- TMA
+      if (lane == 0) {
+        const int ntile = nkt[1] > 0 ? 2 : 1;
+        mbar_expect_tx(bar_q, 3 * kPfSlabBytes * ntile);
+        for (int g = 0; g < ntile; ++g)
+          for (int s = 0; s < 3; ++s)
+            tma_load(sb + kPfQ + (3 * g + s) * kPfSlabBytes, &tm_q, bar_q, h * 192 + 64 * s,
+                     start + q0 + g * kPfTile);
+        int issued_k = 0, issued_v = 0;
+        for (int j = 0; j < nk && ok; ++j) {
+          // the key tile is free once both products of the previous tile are done with it
+          if (j > 0) ok = pf_wait(bar_kfree, (j - 1) & 1, a.err);
+          if (!ok) break;
+          ++issued_k;
+          mbar_expect_tx(bar_k, 3 * kPfSlabBytes);
+          for (int s = 0; s < 2; ++s)
+            tma_load(sb + kPfK + s * kPfSlabBytes, &tm_kn, bar_k, h * 128 + 64 * s,
+                     start + j * kPfTile);
+          tma_load(sb + kPfK + 2 * kPfSlabBytes, &tm_kr, bar_k, r, start + j * kPfTile);
+          if (j > 0) ok = pf_wait(bar_vfree, (j - 1) & 1, a.err);
+          if (!ok) break;
+          ++issued_v;
+          mbar_expect_tx(bar_v, 2 * kPfSlabBytes);
+          for (int s = 0; s < 2; ++s)
+            tma_load(sb + kPfV + s * kPfSlabBytes, &tm_v, bar_v, h * 128 + 64 * s,
+                     start + j * kPfTile);
+        }
+        // the last copies have landed before the CTA may exit (their phases are the barriers'
+        // last, so the wait holds whether or not a consumer saw them)
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try(bar_q, 0) && globaltimer() - t0 < kPfTimeoutNs) {
+        }
+        while (issued_k > 0 && !mbar_try(bar_k, (issued_k - 1) & 1) &&
+               globaltimer() - t0 < 2 * kPfTimeoutNs) {
+        }
+        while (issued_v > 0 && !mbar_try(bar_v, (issued_v - 1) & 1) &&
+               globaltimer() - t0 < 3 * kPfTimeoutNs) {
         }
       }
-      ok = __syncthreads_and(ok);
-      if (!ok) break;
-      ok = pf_wait(bar_s, j & 1, a.err);
-      ok = __syncthreads_and(ok);
-      if (!ok) break;
-      done_s = j + 1;
-      tc_after();
-      // the key buffer is free: the next tile's keys load during this tile's softmax and P . V
-      if (threadIdx.x == 0 && j + 1 < nkt) load_k(j + 1);
-      if (j + 1 < nkt) issued_k = j + 2;
-      uint32_t v[128];
-      tmem_ld128(t_s, v);
-      // causal mask: key k0 + c is visible to query qi when k0 + c <= qi (and inside the
-      // sequence, which qi < len implies)
-      const int k0 = j * kPfTile;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float s = (k0 + c <= qi) ? __uint_as_float(v[c]) * a.c2 : -INFINITY;
-        v[c] = __float_as_uint(s);
-        mx = fmaxf(mx, s);
-      }
-      float alpha = 1.f;
-      if (j == 0) {
-        m_ref = qi < len ? mx : 0.f;  // key 0 is always visible to a query of the sequence
-      } else if (mx > m_ref + 8.f) {
-        alpha = ex2(m_ref - mx);
-        m_ref = mx;
-      }
-      // P in bf16 as the A operand of P . V: row qi, keys in 2 slabs of 64 (128-byte rows
-      // swizzled by row % 8); l sums the bf16 values the MMA consumes
-      float rs = 0.f;
-      const uint32_t prow = sb + kPfP + (uint32_t)threadIdx.x * 128;
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 64 * s + 8 * g + 2 * e;
-            const float p0 = ex2(__uint_as_float(v[c]) - m_ref);
-            const float p1 = ex2(__uint_as_float(v[c + 1]) - m_ref);
-            w4[e] = pack_bf16(p0, p1);
-            rs += __uint_as_float(w4[e] << 16) + __uint_as_float(w4[e] & 0xffff0000u);
+    } else if (warp == 9) {
+      // ---------------------------------------------------------------- MMA issue
+      if (lane == 0) {
+        ok = pf_wait(bar_q, 0, a.err);
+        const uint32_t id_s = idesc(128, 128, 0, 0), id_o = idesc(128, 128, 1);
+        for (int j = 0; j < nk && ok; ++j) {
+          ok = pf_wait(bar_k, j & 1, a.err);
+          for (int g = 0; g < 2 && ok; ++g) {
+            if (j >= nkt[g]) continue;
+            // S_g's columns hold P_g of the previous tile until its P . V is done
+            if (j > 0) ok = pf_wait(bar_o + 8 * g, (j - 1) & 1, a.err);
+            if (!ok) break;
+            tc_after();
+            for (int ks = 0; ks < 12; ++ks) {
+              const uint32_t off = (uint32_t)(ks >> 2) * kPfSlabBytes + 32u * (uint32_t)(ks & 3);
+              mma_ss(tmem + 128 * g, sdesc(sb + kPfQ + 3 * g * kPfSlabBytes + off, 16, 1024, 2),
+                     sdesc(sb + kPfK + off, 16, 1024, 2), id_s, ks > 0 ? 1u : 0u);
+            }
+            tc_commit(bar_s + 8 * g);
           }
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                           prow + s * kPfSlabBytes + 16u * (uint32_t)(g ^ (threadIdx.x & 7))),
-                       "r"(w4[0]), "r"(w4[1]), "r"(w4[2]), "r"(w4[3])
-                       : "memory");
+          if (!ok) break;
+          tc_commit(bar_kfree);  // the key tile is free once both products are done
+          ok = pf_wait(bar_v, j & 1, a.err);
+          for (int g = 0; g < 2 && ok; ++g) {
+            if (j >= nkt[g]) continue;
+            ok = pf_wait(bar_p + 8 * g, j & 1, a.err);
+            if (!ok) break;
+            tc_after();
+            for (int ks = 0; ks < 8; ++ks)  // 16 keys per step: 8 TMEM columns of P
+              mma_ts(tmem + 256 + 128 * g, tmem + 128 * g + 8 * ks,
+                     sdesc(sb + kPfV + 2048u * (uint32_t)ks, kPfSlabBytes, 1024, 2), id_o,
+                     (j > 0 || ks > 0) ? 1u : 0u);
+            tc_commit(bar_o + 8 * g);
+          }
+          if (!ok) break;
+          tc_commit(bar_vfree);
         }
       }
-      l = l * alpha + rs;
-      // TMEM loads and stores are warp-wide: a warp rescales when any of its rows must
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // the previous P . V is complete (waited for below): rescale this row of O
+    } else if (nkt[warp >> 2] > 0) {
+      // ---------------------------------------------------------------- softmax of tile g
+      const int g = warp >> 2, quad = warp & 3;
+      const int row = quad * 32 + lane;          // TMEM lane = query row within the tile
+      const int qi = q0 + g * kPfTile + row;     // query index within the sequence
+      const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+      const uint32_t t_s = tmem + lane_base + 128 * g, t_o = tmem + lane_base + 256 + 128 * g;
+      float m_ref = 0.f, l = 0.f;
+      for (int j = 0; j < nkt[g] && ok; ++j) {
+        ok = warp_all_wait(bar_s + 8 * g, j & 1, a.err);
+        if (!ok) break;
+        tc_after();
+        uint32_t v[128];
+        tmem_ld128(t_s, v);
+        const int k0 = j * kPfTile;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const float s = (k0 + c <= qi) ? __uint_as_float(v[c]) * a.c2 : -INFINITY;
+          v[c] = __float_as_uint(s);
+          mx = fmaxf(mx, s);
+        }
+        float alpha = 1.f;
+        if (j == 0) {
+          m_ref = qi < len ? mx : 0.f;  // key 0 is visible to every query of the sequence
+        } else if (mx > m_ref + 8.f) {
+          alpha = ex2(m_ref - mx);
+          m_ref = mx;
+        }
+        // P in bf16 over the tile's S columns (keys 2c, 2c + 1 in column c); l sums the bf16
+        // values the MMA consumes
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = ex2(__uint_as_float(v[2 * c]) - m_ref);
+          const float p1 = ex2(__uint_as_float(v[2 * c + 1]) - m_ref);
+          v[c] = pack_bf16(p0, p1);
+          rs += __uint_as_float(v[c] << 16) + __uint_as_float(v[c] & 0xffff0000u);
+        }
+        l = l * alpha + rs;
+        // the previous P . V is complete (S_g of this tile was issued after it): rescale O
+        // (TMEM accesses are warp-wide: a warp rescales when any of its rows must)
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c0, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_o + c0, o);
+          }
+        }
+        uint32_t w0[32], w1[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          w0[i] = v[i];
+          w1[i] = v[32 + i];
+        }
+        tmem_st32(t_s, w0);
+        tmem_st32(t_s + 32, w1);
+        tmem_wait_st();
+        tc_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p + 8 * g);
+      }
+      if (ok) ok = warp_all_wait(bar_o + 8 * g, (nkt[g] - 1) & 1, a.err);
+      if (ok) {
+        tc_after();
+        // o = O / l for this thread's query row, bf16 (every lane takes part in the warp-wide
+        // TMEM loads; rows past the sequence end store nothing)
+        const float inv = qi < len ? 1.f / l : 0.f;
+        __nv_bfloat16* dst = a.o + ((size_t)(start + min(qi, len - 1)) * a.H + h) * 128;
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(t_o + c0, o);
+          if (qi < len) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(t_o + c0, o);
-        }
-        tmem_wait_st();
-      }
-      fence_proxy_async();
-      tc_before();
-      __syncthreads();
-      // O += P V_j
-      if (threadIdx.x == 0) {
-        ok = pf_wait(bar_v, j & 1, a.err);
-        if (ok) {
-          tc_after();
-          const uint32_t id = idesc(128, 128, 1);
-          for (int ks = 0; ks < 8; ++ks)  // 16 keys per step; V's two d_v slabs LBO apart
-            mma_ss(tmem + 128, sdesc(sb + kPfP + (uint32_t)(ks >> 2) * kPfSlabBytes + 32u * (ks & 3), 16, 1024, 2),
-                   sdesc(sb + kPfV + 2048u * (uint32_t)ks, kPfSlabBytes, 1024, 2), id,
-                   (j > 0 || ks > 0) ? 1u : 0u);
-          tc_commit(bar_o);
-        }
-      }
-      ok = __syncthreads_and(ok);
-      if (!ok) break;
-      ok = __syncthreads_and(pf_wait(bar_o, j & 1, a.err));
-      if (!ok) break;
-      done_o = j + 1;
-      // values and P are free again
-      if (threadIdx.x == 0 && j + 1 < nkt) load_v(j + 1);
-      if (j + 1 < nkt) issued_v = j + 2;
-    }
-    if (ok) {
-      tc_after();
-      // o = O / l for this thread's query row, bf16 (every lane takes part in the warp-wide
-      // TMEM loads; rows past the sequence end store nothing)
-      const float inv = qi < len ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = a.o + ((size_t)(start + min(qi, len - 1)) * a.H + h) * 128;
-#pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(t_o + c0, o);
-        if (qi < len) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
-            w.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-            w.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-            w.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-            *(uint4*)(dst + c0 + i) = w;
+            for (int i = 0; i < 32; i += 8) {
+              uint4 w;
+              w.x = pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+              w.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+              w.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+              w.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+              *(uint4*)(dst + c0 + i) = w;
+            }
           }
         }
       }
     }
   }
+  __syncwarp();
   tc_before();
   __syncthreads();
   tc_after();
-  if (!ok && threadIdx.x == 0) {
-    // copies that may still land, MMAs that may still run
+  if (threadIdx.x == 9 * 32) {
+    // every MMA issued here (none when the work was empty) is done before TMEM is freed; the
+    // copies issued were all waited for by the MMA thread unless a wait gave up, in which case
+    // the last ones get a bounded wait too
+    tc_commit(bar_fin);
     const uint64_t t0 = globaltimer();
-    while (issued_k > done_s && !mbar_try(bar_k, (issued_k - 1) & 1) &&
-           globaltimer() - t0 < kPfTimeoutNs) {
-    }
-    while (issued_v > done_o && !mbar_try(bar_v, (issued_v - 1) & 1) &&
-           globaltimer() - t0 < 2 * kPfTimeoutNs) {
-    }
-    tc_commit(bar_s);  // completes once every MMA issued so far is done
-    while (!mbar_try(bar_s, done_s & 1) && globaltimer() - t0 < 3 * kPfTimeoutNs) {
+    while (!mbar_try(bar_fin, 0) && globaltimer() - t0 < kPfTimeoutNs) {
     }
   }
   __syncthreads();
@@ -438,10 +476,10 @@ cudaError_t launch_prefill(const mla_config& c, const void* q_nope, const void* 
     e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kPfSmem);
     if (e != cudaSuccess) return e;
-    const int qtiles = (max_seqlen + kPfTile - 1) / kPfTile;
-    PrefillArgs a{cu, (__nv_bfloat16*)o, err, batch, H, qtiles, c2};
-    return launch_pdl(prefill_tc_kernel, dim3(batch * qtiles, H), dim3(128), (size_t)kPfSmem, st,
-                      tq, tkn, tkr, tv, a, r);
+    const int pairs = (max_seqlen + 2 * kPfTile - 1) / (2 * kPfTile);
+    PrefillArgs a{cu, (__nv_bfloat16*)o, err, batch, H, pairs, c2};
+    return launch_pdl(prefill_tc_kernel, dim3(batch * pairs, H), dim3(kPfThreads),
+                      (size_t)kPfSmem, st, tq, tkn, tkr, tv, a, r);
   }
   dim3 grid(n, (H + 3) / 4);
   return bf ? launch_pdl(prefill_simt_kernel<__nv_bfloat16>, grid, dim3(128), 0, st,
