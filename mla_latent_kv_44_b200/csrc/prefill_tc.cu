@@ -272,14 +272,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_after();
         uint32_t v[128];
         tmem_ld128(t_s, v);
-        const int k0 = j * kPfTile;
-        float mx = -INFINITY;
+        // the last key tile is the diagonal one (it starts at the query tile's first row):
+        // keys past the row's query are masked there; earlier tiles are visible whole
+        if (j == nkt[g] - 1) {
+          const int lim = row;  // keys 0 .. row of the tile are visible
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float s = (k0 + c <= qi) ? __uint_as_float(v[c]) * a.c2 : -INFINITY;
-          v[c] = __float_as_uint(s);
-          mx = fmaxf(mx, s);
+          for (int c = 0; c < 128; ++c)
+            if (c > lim) v[c] = 0xff800000u;  // -inf
         }
+        // the row maximum of the raw scores (the scale is positive), four three-input chains
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int k = 0; k < 128; k += 8)
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            mx4[c] = fmax3(mx4[c], __uint_as_float(v[k + 2 * c]), __uint_as_float(v[k + 2 * c + 1]));
+        const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * a.c2;
         float alpha = 1.f;
         if (j == 0) {
           m_ref = qi < len ? mx : 0.f;  // key 0 is visible to every query of the sequence
@@ -287,16 +295,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           alpha = ex2(m_ref - mx);
           m_ref = mx;
         }
-        // P in bf16 over the tile's S columns (keys 2c, 2c + 1 in column c); l sums the bf16
-        // values the MMA consumes
-        float rs = 0.f;
+        // P = exp2(s * c2 - m_ref) in bf16 over the tile's S columns (keys 2c, 2c + 1 in
+        // column c), the argument two at a time in one packed fma; l sums the bf16 values the
+        // MMA consumes, two at a time in packed adds
+        const float2 c2x2 = make_float2(a.c2, a.c2), nm = make_float2(-m_ref, -m_ref);
+        float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2(__uint_as_float(v[2 * c]) - m_ref);
-          const float p1 = ex2(__uint_as_float(v[2 * c + 1]) - m_ref);
-          v[c] = pack_bf16(p0, p1);
-          rs += __uint_as_float(v[c] << 16) + __uint_as_float(v[c] & 0xffff0000u);
+          const float2 x = __ffma2_rn(
+              make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])), c2x2, nm);
+          v[c] = pack_bf16(ex2(x.x), ex2(x.y));
+          rs2[c & 1] = __fadd2_rn(
+              rs2[c & 1], make_float2(__uint_as_float(v[c] << 16), __uint_as_float(v[c] & 0xffff0000u)));
         }
+        const float rs = (rs2[0].x + rs2[1].x) + (rs2[0].y + rs2[1].y);
         l = l * alpha + rs;
         // the previous P . V is complete (S_g of this tile was issued after it): rescale O
         // (TMEM accesses are warp-wide: a warp rescales when any of its rows must)
