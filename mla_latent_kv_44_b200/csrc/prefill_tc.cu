@@ -45,10 +45,14 @@ constexpr int kPfTile = 128;                   // queries per tile = keys per ti
 constexpr int kPfSlabBytes = kPfTile * 128;    // 128 rows x 64 bf16: 16 KB
 constexpr int kPfQ = 0;                        // two query tiles: 3 slabs each (q_nope 0-63,
                                                // 64-127, q_rope)
-constexpr int kPfK = kPfQ + 6 * kPfSlabBytes;  // keys: 3 slabs (K_nope 0-63, 64-127, k_rope)
-constexpr int kPfV = kPfK + 3 * kPfSlabBytes;  // values: 2 slabs (d_v 0-63, 64-127), MN-major
-constexpr int kPfBar = kPfV + 2 * kPfSlabBytes;
-constexpr int kPfSmem = kPfBar + 128 + 1024;
+constexpr int kPfK = kPfQ + 6 * kPfSlabBytes;  // keys: a ring of 4 slabs; key tile j's slab s
+                                               // (K_nope 0-63, 64-127, k_rope) in slot
+                                               // (3j + s) % 4
+constexpr int kPfKSlots = 4;
+constexpr int kPfV = kPfK + kPfKSlots * kPfSlabBytes;  // values: 2 stages of 2 slabs (d_v 0-63,
+                                                       // 64-127), MN-major
+constexpr int kPfBar = kPfV + 4 * kPfSlabBytes;
+constexpr int kPfSmem = kPfBar + 256 + 1024;
 constexpr int kPfThreads = 320;                // warps 0-3, 4-7: softmax of tiles A, B;
                                                // 8: TMA; 9: MMA issue
 constexpr uint32_t kPfTmemCols = 512;          // S_A, S_B, O_A, O_B: 128 columns each
@@ -64,6 +68,55 @@ __device__ __forceinline__ bool pf_wait(uint32_t bar, uint32_t parity, uint32_t*
   }
   return true;
 }
+
+// 2^x for a pair on the FMA pipe, so that the exp2 unit and the FMA pipe share a tile's
+// exponentials: Cody and Waite's reduction x = k + f with k = round(x) and f in [-1/2, 1/2]
+// (k from adding 1.5 * 2^23, which leaves it in the low mantissa bits), 2^f by a cubic fitted
+// to the relative error on [-1/2, 1/2] (at most 7.5e-5, against 2^-9 for the bf16 rounding of
+// P that follows), and k added to the exponent field as an integer. Arguments below -126
+// (masked keys' -inf included) are clamped there; their 2^x is below 2^-125 instead of 0.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 k = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(k, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(f, make_float2(0.05517132f, 0.05517132f),
+                        make_float2(0.24261054f, 0.24261054f));
+  p = __ffma2_rn(p, f, make_float2(0.69326097f, 0.69326097f));
+  p = __ffma2_rn(p, f, make_float2(0.99992812f, 0.99992812f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// tcgen05 issue from a converged warp: every lane runs the issue loop, so the descriptors stay
+// warp-uniform, and elect.sync picks the one lane that issues.
+__device__ __forceinline__ void mma_ss_warp(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t id,
+                                            uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d), "l"(adesc),
+      "l"(bdesc), "r"(id), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_warp(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t id,
+                                            uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d), "r"(a),
+      "l"(bdesc), "r"(id), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void commit_warp(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          bar)
+      : "memory");
+}
+
+// Pairs of a row's 64 whose exponentials go to the FMA pipe: (pair % 8) < kPfFmaEighths.
+constexpr int kPfFmaEighths = 1;
 
 // Warp-wide bounded wait: the same result in every lane.
 __device__ __forceinline__ bool warp_all_wait(uint32_t bar, uint32_t parity, uint32_t* err) {
@@ -147,14 +200,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t sb = saddr(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x / a.pairs, pr = blockIdx.x - b * a.pairs, h = blockIdx.y;
-  // barriers: q, k, v, kfree, vfree, s[2], p[2], o[2], final
-  const uint32_t bar_q = sb + kPfBar, bar_k = bar_q + 8, bar_v = bar_q + 16;
-  const uint32_t bar_kfree = bar_q + 24, bar_vfree = bar_q + 32;
-  const uint32_t bar_s = bar_q + 40, bar_p = bar_q + 56, bar_o = bar_q + 72;
-  const uint32_t bar_fin = bar_q + 88;
-  uint32_t* tmem_slot = (uint32_t*)(smem + kPfBar + 96);
+  // barriers: q, kfull[4], kfree[4], vfull[2], vfree[2], s[2], p[2], o[2], final
+  const uint32_t bar_q = sb + kPfBar, bar_kfull = bar_q + 8, bar_kfree = bar_q + 40;
+  const uint32_t bar_vfull = bar_q + 72, bar_vfree = bar_q + 88;
+  const uint32_t bar_s = bar_q + 104, bar_p = bar_q + 120, bar_o = bar_q + 136;
+  const uint32_t bar_fin = bar_q + 152;
+  uint32_t* tmem_slot = (uint32_t*)(smem + kPfBar + 160);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 12; ++i) mbar_init(bar_q + 8 * i, (i == 7 || i == 8) ? 4 : 1);
+    for (int i = 0; i < 20; ++i) mbar_init(bar_q + 8 * i, (i == 15 || i == 16) ? 4 : 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -182,6 +235,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (nkt[0] > 0) {
     if (warp == 8) {
       // ---------------------------------------------------------------- TMA
+      // in the order the MMA warp consumes them: key tile j's first slab, its values, then its
+      // other two slabs (their slots are freed by the second score product of tile j - 1)
       if (lane == 0) {
         const int ntile = nkt[1] > 0 ? 2 : 1;
         mbar_expect_tx(bar_q, 3 * kPfSlabBytes * ntile);
@@ -189,73 +244,92 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           for (int s = 0; s < 3; ++s)
             tma_load(sb + kPfQ + (3 * g + s) * kPfSlabBytes, &tm_q, bar_q, h * 192 + 64 * s,
                      start + q0 + g * kPfTile);
-        int issued_k = 0, issued_v = 0;
+        int k_issued = 0, v_issued = 0;  // slabs and value tiles issued
+        auto load_k = [&](int j, int sl) {
+          const int u = 3 * j + sl, slot = u & (kPfKSlots - 1);
+          if (u >= kPfKSlots && !pf_wait(bar_kfree + 8 * slot, ((u >> 2) - 1) & 1, a.err))
+            return false;
+          mbar_expect_tx(bar_kfull + 8 * slot, kPfSlabBytes);
+          if (sl < 2)
+            tma_load(sb + kPfK + slot * kPfSlabBytes, &tm_kn, bar_kfull + 8 * slot,
+                     h * 128 + 64 * sl, start + j * kPfTile);
+          else
+            tma_load(sb + kPfK + slot * kPfSlabBytes, &tm_kr, bar_kfull + 8 * slot, r,
+                     start + j * kPfTile);
+          k_issued = u + 1;
+          return true;
+        };
         for (int j = 0; j < nk && ok; ++j) {
-          // the key tile is free once both products of the previous tile are done with it
-          if (j > 0) ok = pf_wait(bar_kfree, (j - 1) & 1, a.err);
+          ok = load_k(j, 0);
           if (!ok) break;
-          ++issued_k;
-          mbar_expect_tx(bar_k, 3 * kPfSlabBytes);
-          for (int s = 0; s < 2; ++s)
-            tma_load(sb + kPfK + s * kPfSlabBytes, &tm_kn, bar_k, h * 128 + 64 * s,
-                     start + j * kPfTile);
-          tma_load(sb + kPfK + 2 * kPfSlabBytes, &tm_kr, bar_k, r, start + j * kPfTile);
-          if (j > 0) ok = pf_wait(bar_vfree, (j - 1) & 1, a.err);
+          const int vs = j & 1;
+          if (j >= 2) ok = pf_wait(bar_vfree + 8 * vs, ((j >> 1) - 1) & 1, a.err);
           if (!ok) break;
-          ++issued_v;
-          mbar_expect_tx(bar_v, 2 * kPfSlabBytes);
+          mbar_expect_tx(bar_vfull + 8 * vs, 2 * kPfSlabBytes);
           for (int s = 0; s < 2; ++s)
-            tma_load(sb + kPfV + s * kPfSlabBytes, &tm_v, bar_v, h * 128 + 64 * s,
-                     start + j * kPfTile);
+            tma_load(sb + kPfV + (2 * vs + s) * kPfSlabBytes, &tm_v, bar_vfull + 8 * vs,
+                     h * 128 + 64 * s, start + j * kPfTile);
+          v_issued = j + 1;
+          ok = load_k(j, 1) && load_k(j, 2);
         }
-        // the last copies have landed before the CTA may exit (their phases are the barriers'
-        // last, so the wait holds whether or not a consumer saw them)
+        // the last copies have landed before the CTA may exit (each barrier's last armed phase
+        // is its last, so the wait holds whether or not a consumer saw it)
         const uint64_t t0 = globaltimer();
         while (!mbar_try(bar_q, 0) && globaltimer() - t0 < kPfTimeoutNs) {
         }
-        while (issued_k > 0 && !mbar_try(bar_k, (issued_k - 1) & 1) &&
-               globaltimer() - t0 < 2 * kPfTimeoutNs) {
-        }
-        while (issued_v > 0 && !mbar_try(bar_v, (issued_v - 1) & 1) &&
-               globaltimer() - t0 < 3 * kPfTimeoutNs) {
-        }
+        for (int u = max(0, k_issued - kPfKSlots); u < k_issued; ++u)
+          while (!mbar_try(bar_kfull + 8 * (u & (kPfKSlots - 1)), (u >> 2) & 1) &&
+                 globaltimer() - t0 < 2 * kPfTimeoutNs) {
+          }
+        for (int j = max(0, v_issued - 2); j < v_issued; ++j)
+          while (!mbar_try(bar_vfull + 8 * (j & 1), (j >> 1) & 1) &&
+                 globaltimer() - t0 < 3 * kPfTimeoutNs) {
+          }
       }
     } else if (warp == 9) {
       // ---------------------------------------------------------------- MMA issue
-      if (lane == 0) {
-        ok = pf_wait(bar_q, 0, a.err);
+      // Per key tile j: O_A += P_A V_j, S_A = Q_A K_{j+1}^T, O_B += P_B V_j, S_B = Q_B K_{j+1}^T,
+      // so that each tile's next scores are computed while the other tile's softmax runs. The
+      // whole warp runs the loop and waits warp-wide; one elected lane issues.
+      {
         const uint32_t id_s = idesc(128, 128, 0, 0), id_o = idesc(128, 128, 1);
-        for (int j = 0; j < nk && ok; ++j) {
-          ok = pf_wait(bar_k, j & 1, a.err);
-          for (int g = 0; g < 2 && ok; ++g) {
-            if (j >= nkt[g]) continue;
-            // S_g's columns hold P_g of the previous tile until its P . V is done
-            if (j > 0) ok = pf_wait(bar_o + 8 * g, (j - 1) & 1, a.err);
-            if (!ok) break;
+        // S_g = Q_g K_j^T; the last product to read key tile j frees its slabs one by one
+        auto scores = [&](int g, int j) {
+          const bool last = g == 1 || nkt[1] <= j;
+          for (int sl = 0; sl < 3; ++sl) {
+            const int u = 3 * j + sl, slot = u & (kPfKSlots - 1);
+            if (!warp_all_wait(bar_kfull + 8 * slot, (u >> 2) & 1, a.err)) return false;
             tc_after();
-            for (int ks = 0; ks < 12; ++ks) {
-              const uint32_t off = (uint32_t)(ks >> 2) * kPfSlabBytes + 32u * (uint32_t)(ks & 3);
-              mma_ss(tmem + 128 * g, sdesc(sb + kPfQ + 3 * g * kPfSlabBytes + off, 16, 1024, 2),
-                     sdesc(sb + kPfK + off, 16, 1024, 2), id_s, ks > 0 ? 1u : 0u);
-            }
-            tc_commit(bar_s + 8 * g);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss_warp(tmem + 128 * g,
+                          sdesc(sb + kPfQ + (3 * g + sl) * kPfSlabBytes + 32u * kk, 16, 1024, 2),
+                          sdesc(sb + kPfK + slot * kPfSlabBytes + 32u * kk, 16, 1024, 2), id_s,
+                          (sl | kk) ? 1u : 0u);
+            if (last) commit_warp(bar_kfree + 8 * slot);
           }
-          if (!ok) break;
-          tc_commit(bar_kfree);  // the key tile is free once both products are done
-          ok = pf_wait(bar_v, j & 1, a.err);
+          commit_warp(bar_s + 8 * g);
+          return true;
+        };
+        ok = warp_all_wait(bar_q, 0, a.err) && scores(0, 0) && (nkt[1] == 0 || scores(1, 0));
+        for (int j = 0; j < nk && ok; ++j) {
+          const int vs = j & 1;
+          ok = warp_all_wait(bar_vfull + 8 * vs, (j >> 1) & 1, a.err);
           for (int g = 0; g < 2 && ok; ++g) {
             if (j >= nkt[g]) continue;
-            ok = pf_wait(bar_p + 8 * g, j & 1, a.err);
+            ok = warp_all_wait(bar_p + 8 * g, j & 1, a.err);
             if (!ok) break;
             tc_after();
             for (int ks = 0; ks < 8; ++ks)  // 16 keys per step: 8 TMEM columns of P
-              mma_ts(tmem + 256 + 128 * g, tmem + 128 * g + 8 * ks,
-                     sdesc(sb + kPfV + 2048u * (uint32_t)ks, kPfSlabBytes, 1024, 2), id_o,
-                     (j > 0 || ks > 0) ? 1u : 0u);
-            tc_commit(bar_o + 8 * g);
+              mma_ts_warp(tmem + 256 + 128 * g, tmem + 128 * g + 8 * ks,
+                          sdesc(sb + kPfV + 2 * vs * kPfSlabBytes + 2048u * (uint32_t)ks,
+                                kPfSlabBytes, 1024, 2),
+                          id_o, (j > 0 || ks > 0) ? 1u : 0u);
+            commit_warp(bar_o + 8 * g);
+            if (g == 1 || nkt[1] <= j) commit_warp(bar_vfree + 8 * vs);  // V_j's last reader
+            // S_g's columns hold P_g until its P . V is done
+            if (j + 1 < nkt[g])
+              ok = warp_all_wait(bar_o + 8 * g, j & 1, a.err) && scores(g, j + 1);
           }
-          if (!ok) break;
-          tc_commit(bar_vfree);
         }
       }
     } else if (nkt[warp >> 2] > 0) {
@@ -296,15 +370,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           m_ref = mx;
         }
         // P = exp2(s * c2 - m_ref) in bf16 over the tile's S columns (keys 2c, 2c + 1 in
-        // column c), the argument two at a time in one packed fma; l sums the bf16 values the
-        // MMA consumes, two at a time in packed adds
+        // column c), the argument two at a time in one packed fma, a quarter of the pairs'
+        // exponentials on the FMA pipe; l sums the bf16 values the MMA consumes, two at a time
+        // in packed adds
         const float2 c2x2 = make_float2(a.c2, a.c2), nm = make_float2(-m_ref, -m_ref);
         float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const float2 x = __ffma2_rn(
               make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])), c2x2, nm);
-          v[c] = pack_bf16(ex2(x.x), ex2(x.y));
+          const float2 e = (c & 7) < kPfFmaEighths ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
+          v[c] = pack_bf16(e.x, e.y);
           rs2[c & 1] = __fadd2_rn(
               rs2[c & 1], make_float2(__uint_as_float(v[c] << 16), __uint_as_float(v[c] & 0xffff0000u)));
         }
