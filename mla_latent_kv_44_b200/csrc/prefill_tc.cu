@@ -457,6 +457,192 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                  : "memory");
 }
 
+// K_nope = c_kv W_UK^T and V = c_kv W_UV^T for every prompt token on the tensor cores, one
+// GEMM with M = 128 tokens, N = 128 weight rows, K = r per tile. A persistent CTA per SM walks
+// work items (a 128-row weight tile, a chunk of token tiles): the weight tile stays in shared
+// memory (r / 64 slabs of 16 KB, each replaced for the next item as soon as the item's last
+// products are done with it) while the tokens' c_kv slabs stream through a ring; two TMEM
+// accumulators let the epilogue of one token tile (bf16, a thread per token writing the tile's
+// 128 contiguous outputs) overlap the products of the next. Warps: 0 TMA, 1 MMA issue (whole
+// warp, one elected lane), 2-5 epilogue.
+constexpr int kExSlab = 128 * 128;             // 128 rows x 64 bf16: 16 KB
+constexpr int kExMaxSlabs = 8;                 // resident weight tile: r <= 512
+constexpr int kExStages = 6;                   // token slabs in flight
+constexpr int kExW = 0;
+constexpr int kExX = kExW + kExMaxSlabs * kExSlab;
+constexpr int kExBar = kExX + kExStages * kExSlab;
+constexpr int kExSmem = kExBar + 512 + 1024;
+constexpr int kExThreads = 192;
+constexpr int kExChunk = 16;                   // token tiles per work item
+
+struct ExpandArgs {
+  __nv_bfloat16* kn;
+  __nv_bfloat16* v;
+  uint32_t* err;
+  int n;              // tokens
+  int ksl;            // 64-wide slabs of r
+  int mt_k, mtiles;   // 128-row weight tiles of W_UK; of W_UK and W_UV together
+  int chunks, items;  // token chunks per weight tile; work items
+  int ldk, ldv;       // output row pitches (elements)
+};
+
+__global__ void __launch_bounds__(kExThreads)
+expand_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wk,
+                 const __grid_constant__ CUtensorMap tm_wv, const ExpandArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sb = saddr(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // barriers: wfull[8], wfree[8], xfull[6], xfree[6], afull[2], afree[2], final
+  const uint32_t bar_wfull = sb + kExBar, bar_wfree = bar_wfull + 8 * kExMaxSlabs;
+  const uint32_t bar_xfull = bar_wfree + 8 * kExMaxSlabs, bar_xfree = bar_xfull + 8 * kExStages;
+  const uint32_t bar_afull = bar_xfree + 8 * kExStages, bar_afree = bar_afull + 16;
+  const uint32_t bar_fin = bar_afree + 16;
+  uint32_t* tmem_slot = (uint32_t*)(smem + kExBar + 320);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2 * kExMaxSlabs + 2 * kExStages + 4 + 1; ++i) {
+      const uint32_t b = bar_wfull + 8 * i;
+      mbar_init(b, (b == bar_afree || b == bar_afree + 8) ? 4 : 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     saddr(tmem_slot)),
+                 "r"(256)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  const uint32_t tmem = *tmem_slot;
+  wait_prior_grid();
+  const int ttiles = (a.n + 127) / 128;
+  bool ok = true;
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      int kx = 0, li = 0;
+      for (int it = blockIdx.x; it < a.items && ok; it += gridDim.x, ++li) {
+        const int mt = it / a.chunks, tt0 = (it - mt * a.chunks) * kExChunk;
+        const int tt1 = min(ttiles, tt0 + kExChunk);
+        const bool uk = mt < a.mt_k;
+        for (int tt = tt0; tt < tt1 && ok; ++tt)
+          for (int s = 0; s < a.ksl; ++s, ++kx) {
+            if (tt == tt0) {
+              // weight slab s, once the previous item's last products are done with it
+              if (li > 0 && !pf_wait(bar_wfree + 8 * s, (li - 1) & 1, a.err)) {
+                ok = false;
+                break;
+              }
+              mbar_expect_tx(bar_wfull + 8 * s, kExSlab);
+              tma_load(sb + kExW + s * kExSlab, uk ? &tm_wk : &tm_wv, bar_wfull + 8 * s, 64 * s,
+                       (uk ? mt : mt - a.mt_k) * 128);
+            }
+            const int st = kx % kExStages, use = kx / kExStages;
+            if (use > 0 && !pf_wait(bar_xfree + 8 * st, (use - 1) & 1, a.err)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(bar_xfull + 8 * st, kExSlab);
+            tma_load(sb + kExX + st * kExSlab, &tm_x, bar_xfull + 8 * st, 64 * s, tt * 128);
+          }
+      }
+      // the last copies have landed before the CTA may exit
+      const uint64_t t0 = globaltimer();
+      for (int s = 0; s < a.ksl && li > 0; ++s)
+        while (!mbar_try(bar_wfull + 8 * s, (li - 1) & 1) && globaltimer() - t0 < kPfTimeoutNs) {
+        }
+      for (int u = max(0, kx - kExStages); u < kx; ++u)
+        while (!mbar_try(bar_xfull + 8 * (u % kExStages), (u / kExStages) & 1) &&
+               globaltimer() - t0 < 2 * kPfTimeoutNs) {
+        }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue
+    const uint32_t id = idesc(128, 128, 0, 0);
+    int kx = 0, tcount = 0, li = 0;
+    for (int it = blockIdx.x; it < a.items && ok; it += gridDim.x, ++li) {
+      const int mt = it / a.chunks, tt0 = (it - mt * a.chunks) * kExChunk;
+      const int tt1 = min(ttiles, tt0 + kExChunk);
+      for (int tt = tt0; tt < tt1 && ok; ++tt, ++tcount) {
+        const int acc = tcount & 1;
+        // the accumulator's previous tile has been read out by the epilogue
+        if (tcount >= 2) ok = warp_all_wait(bar_afree + 8 * acc, ((tcount >> 1) - 1) & 1, a.err);
+        for (int s = 0; s < a.ksl && ok; ++s, ++kx) {
+          const int st = kx % kExStages;
+          if (tt == tt0) ok = warp_all_wait(bar_wfull + 8 * s, li & 1, a.err);
+          ok = ok && warp_all_wait(bar_xfull + 8 * st, (kx / kExStages) & 1, a.err);
+          if (!ok) break;
+          tc_after();
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss_warp(tmem + 128 * acc, sdesc(sb + kExX + st * kExSlab + 32u * kk, 16, 1024, 2),
+                        sdesc(sb + kExW + s * kExSlab + 32u * kk, 16, 1024, 2), id,
+                        (s | kk) ? 1u : 0u);
+          commit_warp(bar_xfree + 8 * st);
+          if (tt == tt1 - 1) commit_warp(bar_wfree + 8 * s);  // the item's last read of slab s
+        }
+        if (ok) commit_warp(bar_afull + 8 * acc);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    int tcount = 0;
+    for (int it = blockIdx.x; it < a.items && ok; it += gridDim.x) {
+      const int mt = it / a.chunks, tt0 = (it - mt * a.chunks) * kExChunk;
+      const int tt1 = min(ttiles, tt0 + kExChunk);
+      const bool uk = mt < a.mt_k;
+      __nv_bfloat16* out = uk ? a.kn : a.v;
+      const int ld = uk ? a.ldk : a.ldv, col0 = (uk ? mt : mt - a.mt_k) * 128;
+      for (int tt = tt0; tt < tt1 && ok; ++tt, ++tcount) {
+        const int acc = tcount & 1;
+        ok = warp_all_wait(bar_afull + 8 * acc, (tcount >> 1) & 1, a.err);
+        if (!ok) break;
+        tc_after();
+        const int token = tt * 128 + quad * 32 + lane;
+        __nv_bfloat16* dst = out + (size_t)min(token, a.n - 1) * ld + col0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t x[32];
+          tmem_ld32(tmem + lane_base + 128 * acc + c0, x);
+          if (token < a.n) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 w;
+              w.x = pack_bf16(__uint_as_float(x[i]), __uint_as_float(x[i + 1]));
+              w.y = pack_bf16(__uint_as_float(x[i + 2]), __uint_as_float(x[i + 3]));
+              w.z = pack_bf16(__uint_as_float(x[i + 4]), __uint_as_float(x[i + 5]));
+              w.w = pack_bf16(__uint_as_float(x[i + 6]), __uint_as_float(x[i + 7]));
+              *(uint4*)(dst + c0 + i) = w;
+            }
+          }
+        }
+        tc_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_afree + 8 * acc);
+      }
+    }
+  }
+  __syncwarp();
+  tc_before();
+  __syncthreads();
+  tc_after();
+  if (threadIdx.x == 32) {
+    // every MMA issued here is done before TMEM is freed
+    tc_commit(bar_fin);
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try(bar_fin, 0) && globaltimer() - t0 < kPfTimeoutNs) {
+    }
+  }
+  __syncthreads();
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256)
+                 : "memory");
+}
+
 // CUDA-core prefill: a warp per (query, head); lanes split the score's dims and the value's.
 template <typename T>
 __global__ void __launch_bounds__(128)
@@ -504,6 +690,13 @@ bool prefill_tc_supported(const mla_config& c) {
          c.kv_rank % 8 == 0;
 }
 
+// The expansion's tensor-core GEMM: bf16, the weight tile resident (r <= 512), whole 128-row
+// weight tiles.
+bool expand_tc_supported(const mla_config& c) {
+  return prefill_tc_supported(c) && c.kv_rank <= 64 * kExMaxSlabs &&
+         (c.num_heads * c.head_dim) % 128 == 0 && (c.num_heads * c.head_dim_v) % 128 == 0;
+}
+
 // Workspace: Q (n, H, d_h + d_r), K_nope (n, H * d_h), V (n, H * d_v) in dtype, then the
 // expansion's partial sums.
 struct PrefillLayout {
@@ -545,11 +738,32 @@ cudaError_t launch_prefill(const mla_config& c, const void* q_nope, const void* 
                                   dh, dr, c.rope_base);
   if (e != cudaSuccess) return e;
   // K_nope and V from c_kv (the first r values of each cache row)
-  const void* wts[2] = {w_uk, w_uv};
-  const int wrows[2] = {H * dh, H * dv};
-  void* outs[2] = {kn, v};
-  e = launch_front_linear(c, rows, n, r, r + dr, wts, wrows, outs, 2, -1, nullptr, 0.f,
-                          w8 + L.part, err, st);
+  if (expand_tc_supported(c)) {
+    CUtensorMap tx, twk, twv;
+    if (!make_bf16_map(&tx, rows, (uint64_t)r, (uint64_t)n, (uint64_t)(r + dr) * 2, 128) ||
+        !make_bf16_map(&twk, w_uk, (uint64_t)r, (uint64_t)H * dh, (uint64_t)r * 2, 128) ||
+        !make_bf16_map(&twv, w_uv, (uint64_t)r, (uint64_t)H * dv, (uint64_t)r * 2, 128))
+      return cudaErrorInvalidValue;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return e;
+    e = cudaFuncSetAttribute(expand_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kExSmem);
+    if (e != cudaSuccess) return e;
+    const int ttiles = (n + 127) / 128, chunks = (ttiles + kExChunk - 1) / kExChunk;
+    const int mt_k = H * dh / 128, mtiles = mt_k + H * dv / 128;
+    ExpandArgs ea{(__nv_bfloat16*)kn, (__nv_bfloat16*)v, err, n, (r + 63) / 64, mt_k, mtiles,
+                  chunks, mtiles * chunks, H * dh, H * dv};
+    e = launch_pdl(expand_tc_kernel, dim3(std::min(sms, ea.items)), dim3(kExThreads),
+                   (size_t)kExSmem, st, tx, twk, twv, ea);
+  } else {
+    const void* wts[2] = {w_uk, w_uv};
+    const int wrows[2] = {H * dh, H * dv};
+    void* outs[2] = {kn, v};
+    e = launch_front_linear(c, rows, n, r, r + dr, wts, wrows, outs, 2, -1, nullptr, 0.f,
+                            w8 + L.part, err, st);
+  }
   if (e != cudaSuccess) return e;
   const float c2 = c.softmax_scale * 1.4426950408889634f;
   if (prefill_tc_supported(c)) {

@@ -64,8 +64,9 @@ def test_prefill_validates_arguments(mla):
     assert call(q) == mla.MLA_ERR_INVALID_ARG
 
 
-def _run(mla, w, lens, seed=5):
-    """Device prefill of sequences of the given lengths, and the oracle's outputs."""
+def _run(mla, w, lens, seed=5, sample=None):
+    """Device prefill of sequences of the given lengths, and the oracle's outputs (for the
+    query tokens sample[b] of sequence b when a sample is given, else for every token)."""
     H, dh, dr, dv, r = w.num_heads, w.head_dim, w.rope_dim, w.head_dim_v, w.kv_rank
     wuk, wuv = (mi.storage_round(w, x) for x in mi.up_projection_weights(w, seed))
     gamma = mi.rms_gain(w, seed, perturbed=True)
@@ -79,10 +80,14 @@ def _run(mla, w, lens, seed=5):
         # the operands as the device holds them: bf16 for a bf16 prefill
         stored = ref.round_bf16 if w.dtype == "bf16" else (lambda x: x)
         Q = stored(np.concatenate([q1, ref.rope_rotate(q2, p[:, None], w.rope_base)], -1))
-        K = np.concatenate([stored(np.einsum("lr,hdr->lhd", rw[:, :r], wuk)),
+        K = np.concatenate([stored(np.einsum("lr,hdr->lhd", rw[:, :r], wuk, optimize=True)),
                             np.repeat(rw[:, None, r:], H, axis=1)], -1)
-        V = stored(np.einsum("lr,hdr->lhd", rw[:, :r], wuv))
-        e = ref.expanded_attention(Q, K, V, w.softmax_scale)
+        V = stored(np.einsum("lr,hdr->lhd", rw[:, :r], wuv, optimize=True))
+        if sample is None:
+            e = ref.expanded_attention(Q, K, V, w.softmax_scale)
+        else:  # token t attends rows 0 .. t: the last query of the prefix t + 1
+            e = np.concatenate([ref.expanded_attention(Q[t:t + 1], K[:t + 1], V[:t + 1],
+                                                       w.softmax_scale) for t in sample[b]])
         qn.append(q1), qr.append(q2), rows.append(rw), pos.append(p), exp.append(e)
     cfg = _cfg(mla, w)
     tdt = cfg.torch_dtype
@@ -124,3 +129,24 @@ def test_prefill_matches_the_oracle(mla, name, lens):
             worst = max(worst, err)
             assert ok, f"sequence {b} (length {lens[b]}), token {t}: error {err:.3g}"
     print(f"{name} {lens}: worst scaled error {worst:.3g}")
+
+
+@pytest.mark.gpu
+def test_prefill_long_prompts_sampled(mla):
+    """Prompts of 2300 and 200 tokens (20 token tiles: the expansion's weight tiles walk two
+    token chunks; nine query-tile pairs): query tokens at tile and chunk boundaries, the
+    first and the last, against the oracle's attention over each token's prefix."""
+    w = mi.WORKLOADS["dsv2"]
+    lens = [2300, 200]
+    sample = [[0, 1, 127, 128, 255, 256, 1000, 2047, 2048, 2049, 2175, 2299],
+              [0, 63, 127, 128, 199]]
+    got, exp = _run(mla, w, lens, sample=sample)
+    worst = 0.0
+    for b in range(len(lens)):
+        assert np.all(np.isfinite(got[b])), f"sequence {b}: non-finite output"
+        for i, t in enumerate(sample[b]):
+            ok, err = compare.within(got[b][t], exp[b][i], w.dtype,
+                                     out_ulps=compare.PROMPT_OUTPUT_ULPS)
+            worst = max(worst, err)
+            assert ok, f"sequence {b}, token {t}: error {err:.3g}"
+    print(f"long prompts {lens}: worst scaled error {worst:.3g}")
