@@ -146,21 +146,23 @@ __device__ __forceinline__ int seq_of(const int32_t* cu, int batch, int i) {
 
 // Q = [q_nope ‖ RoPE(q_rope, pos)] per (token, head): grid (tokens), 16-byte pieces (VEC
 // values) per thread: q_nope pieces copied, q_rope pieces rotated pair by pair (angle and
-// rotation in double, rounded once).
+// rotation in double, rounded once). With rope_only, q holds just the rotated RoPE part
+// (n, H, d_r): the tensor-core attention reads q_nope where the caller keeps it.
 template <typename T>
 __global__ void __launch_bounds__(256)
 prefill_pack_kernel(const T* q_nope, const T* q_rope, const int32_t* pos, T* q, int H, int dh,
-                    int dr, float base) {
+                    int dr, float base, bool rope_only) {
   constexpr int VEC = 16 / sizeof(T);
   extern __shared__ double cs[];  // [2][dr / 2]: cos, sin of the token's angles
-  const int n = blockIdx.x, half = dr / 2, D = dh + dr;
-  const int pn = dh / VEC, pr = dr / VEC, pd = pn + pr;  // pieces per head
+  const int n = blockIdx.x, half = dr / 2;
+  const int pn = dh / VEC, pr = dr / VEC;  // pieces per head
+  const int skip = rope_only ? pn : 0, pd = pn + pr - skip, D = rope_only ? dr : dh + dr;
   wait_prior_grid();
   for (int i = threadIdx.x; i < half; i += blockDim.x)
     rope_cos_sin(pos[n], i, dr, base, &cs[i], &cs[half + i]);
   __syncthreads();
   for (int e = threadIdx.x; e < H * pd; e += blockDim.x) {
-    const int h = e / pd, c = e - h * pd;
+    const int h = e / pd, c = e - h * pd + skip;
     uint4 out;
     if (c < pn) {
       out = *(const uint4*)(q_nope + ((size_t)n * H + h) * dh + c * VEC);
@@ -177,7 +179,7 @@ prefill_pack_kernel(const T* q_nope, const T* q_rope, const int32_t* pos, T* q, 
         y[u + 1] = from_f32<T>((float)(x0 * cs[half + i] + x1 * cs[i]));
       }
     }
-    *(uint4*)(q + ((size_t)n * H + h) * D + c * VEC) = out;
+    *(uint4*)(q + ((size_t)n * H + h) * D + (c - skip) * VEC) = out;
   }
 }
 
@@ -189,17 +191,21 @@ struct PrefillArgs {
   float c2;             // softmax scale * log2(e)
 };
 
-// Grid (batch * pairs, H); 320 threads. TMA maps: q (n, H * 192), kn (n, H * 128),
-// rows (n, r + 64): k_rope at column r, v (n, H * 128); all with 128-row boxes of 64 columns.
+// Grid (batch * pairs, H); 320 threads. TMA maps: qn (n, H * 128) the caller's q_nope, qr
+// (n, H * 64) the rotated RoPE query, kn (n, H * 128), rows (n, r + 64): k_rope at column r,
+// v (n, H * 128); all with 128-row boxes of 64 columns.
 __global__ void __launch_bounds__(kPfThreads)
-prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kn,
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_qr,
+                  const __grid_constant__ CUtensorMap tm_kn,
                   const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_v,
                   const PrefillArgs a, int r) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sb = saddr(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.x / a.pairs, pr = blockIdx.x - b * a.pairs, h = blockIdx.y;
+  // a sequence's pairs of query tiles, longest first, so that the grid's last CTAs are short
+  const int b = blockIdx.x / a.pairs, pr = a.pairs - 1 - (blockIdx.x - b * a.pairs);
+  const int h = blockIdx.y;
   // barriers: q, kfull[4], kfree[4], vfull[2], vfree[2], s[2], p[2], o[2], final
   const uint32_t bar_q = sb + kPfBar, bar_kfull = bar_q + 8, bar_kfree = bar_q + 40;
   const uint32_t bar_vfull = bar_q + 72, bar_vfree = bar_q + 88;
@@ -242,8 +248,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_expect_tx(bar_q, 3 * kPfSlabBytes * ntile);
         for (int g = 0; g < ntile; ++g)
           for (int s = 0; s < 3; ++s)
-            tma_load(sb + kPfQ + (3 * g + s) * kPfSlabBytes, &tm_q, bar_q, h * 192 + 64 * s,
-                     start + q0 + g * kPfTile);
+            tma_load(sb + kPfQ + (3 * g + s) * kPfSlabBytes, s < 2 ? &tm_qn : &tm_qr, bar_q,
+                     s < 2 ? h * 128 + 64 * s : h * 64, start + q0 + g * kPfTile);
         int k_issued = 0, v_issued = 0;  // slabs and value tiles issued
         auto load_k = [&](int j, int sl) {
           const int u = 3 * j + sl, slot = u & (kPfKSlots - 1);
@@ -727,15 +733,15 @@ cudaError_t launch_prefill(const mla_config& c, const void* q_nope, const void* 
   void* q = w8 + L.q;
   void* kn = w8 + L.kn;
   void* v = w8 + L.v;
-  const bool bf = c.dtype == MLA_BF16;
-  // the packed, rotated query
+  const bool bf = c.dtype == MLA_BF16, tc = prefill_tc_supported(c);
+  // the rotated query: its RoPE part alone for the tensor cores, else packed with q_nope
   const size_t csm = (size_t)std::max(1, dr / 2) * 2 * sizeof(double);
   cudaError_t e = bf ? launch_pdl(prefill_pack_kernel<__nv_bfloat16>, dim3(n), dim3(256), csm, st,
                                   (const __nv_bfloat16*)q_nope, (const __nv_bfloat16*)q_rope, pos,
-                                  (__nv_bfloat16*)q, H, dh, dr, c.rope_base)
+                                  (__nv_bfloat16*)q, H, dh, dr, c.rope_base, tc)
                      : launch_pdl(prefill_pack_kernel<float>, dim3(n), dim3(256), csm, st,
                                   (const float*)q_nope, (const float*)q_rope, pos, (float*)q, H,
-                                  dh, dr, c.rope_base);
+                                  dh, dr, c.rope_base, false);
   if (e != cudaSuccess) return e;
   // K_nope and V from c_kv (the first r values of each cache row)
   if (expand_tc_supported(c)) {
@@ -766,10 +772,11 @@ cudaError_t launch_prefill(const mla_config& c, const void* q_nope, const void* 
   }
   if (e != cudaSuccess) return e;
   const float c2 = c.softmax_scale * 1.4426950408889634f;
-  if (prefill_tc_supported(c)) {
-    CUtensorMap tq, tkn, tkr, tv;
-    if (!make_bf16_map(&tq, q, (uint64_t)H * (dh + dr), (uint64_t)n, (uint64_t)H * (dh + dr) * 2,
+  if (tc) {
+    CUtensorMap tqn, tqr, tkn, tkr, tv;
+    if (!make_bf16_map(&tqn, q_nope, (uint64_t)H * dh, (uint64_t)n, (uint64_t)H * dh * 2,
                        kPfTile) ||
+        !make_bf16_map(&tqr, q, (uint64_t)H * dr, (uint64_t)n, (uint64_t)H * dr * 2, kPfTile) ||
         !make_bf16_map(&tkn, kn, (uint64_t)H * dh, (uint64_t)n, (uint64_t)H * dh * 2, kPfTile) ||
         !make_bf16_map(&tkr, rows, (uint64_t)(r + dr), (uint64_t)n, (uint64_t)(r + dr) * 2,
                        kPfTile) ||
@@ -781,7 +788,7 @@ cudaError_t launch_prefill(const mla_config& c, const void* q_nope, const void* 
     const int pairs = (max_seqlen + 2 * kPfTile - 1) / (2 * kPfTile);
     PrefillArgs a{cu, (__nv_bfloat16*)o, err, batch, H, pairs, c2};
     return launch_pdl(prefill_tc_kernel, dim3(batch * pairs, H), dim3(kPfThreads),
-                      (size_t)kPfSmem, st, tq, tkn, tkr, tv, a, r);
+                      (size_t)kPfSmem, st, tqn, tqr, tkn, tkr, tv, a, r);
   }
   dim3 grid(n, (H + 3) / 4);
   return bf ? launch_pdl(prefill_simt_kernel<__nv_bfloat16>, grid, dim3(128), 0, st,
