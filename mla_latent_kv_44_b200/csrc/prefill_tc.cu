@@ -6,20 +6,23 @@
 //                                                                         K and V rebuilt from
 // the latent, the causal mask over the S > 1 new tokens). With many queries per key the
 // expanded form costs fewer FLOPs than the absorbed one (d_h + d_r = 192 per score against
-// r + d_r = 576), so K and V are expanded once per key: one split-K weight-stream launch of the
-// front end's kernel (W_UK and W_UV as two segments, c_kv read in place from the cache rows).
-// A pack kernel writes the query as [q_nope ‖ RoPE(q_rope)] (angles in double).
+// r + d_r = 576), so K and V are expanded once per key, by a persistent tensor-core GEMM that
+// keeps a 128-row weight tile in shared memory and streams the tokens' c_kv (read in place
+// from the cache rows); other shapes use the front end's split-K weight stream. A pack kernel
+// rotates the query's RoPE part (angles in double); the attention reads q_nope where the
+// caller keeps it.
 // The attention kernel takes one CTA per (two adjacent 128-query tiles A and B, head) of a
-// sequence (DeepSeek-V2's head shape: d_h = 128, d_r = 64, d_v = 128, bf16). Both query tiles
-// stay in shared memory and share every key and value tile TMA brings (K_nope of the head and
-// the shared k_rope: three 64-wide slabs; V: two). One thread issues S_A = Q_A K^T and
-// S_B = Q_B K^T (M = 128 queries, N = 128 keys, 12 K-steps) into their TMEM columns, and
-// O_x += P_x V as each tile's P is ready (N = 128, V MN-major, P read from TMEM: the TS form).
-// Two groups of four warps take a tile each (a thread per query row): row maximum, rescale of
-// O in TMEM when the maximum grows by more than 2^8 (exp2 units), P in bf16 written back over
-// the tile's S columns. While one group's softmax runs the tensor core works on the other
-// tile, so the two alternate. Key tiles above a query tile's diagonal are skipped; the
-// diagonal tile is masked. Other shapes and fp32 take a
+// sequence (DeepSeek-V2's head shape: d_h = 128, d_r = 64, d_v = 128, bf16), longest pairs
+// first. Both query tiles stay in shared memory and share every key and value tile TMA brings
+// (K_nope of the head and the shared k_rope: three 64-wide slabs through a ring of four; V: two
+// slabs, double-buffered). One MMA warp issues, per key tile j, O_A += P_A V_j,
+// S_A = Q_A K_{j+1}^T, O_B += P_B V_j, S_B = Q_B K_{j+1}^T (M = 128 queries, N = 128 keys or
+// values; S from shared memory, P read from TMEM: the TS form), the whole warp waiting and one
+// elected lane issuing. Two groups of four warps take a tile each (a thread per query row):
+// row maximum, rescale of O in TMEM when the maximum grows by more than 2^8, exp2 (one pair in
+// eight on the FMA pipe), P in bf16 written back over the tile's S columns. While one group's
+// softmax runs the tensor core works on the other tile's products. Key tiles above a query
+// tile's diagonal are skipped; the diagonal tile is masked. Other shapes and fp32 take a
 // CUDA-core kernel (a warp per (query, head), online softmax over the keys).
 // Every mbarrier wait gives up after 1 s: the kernel then sets MLA_DEV_WAIT_TIMEOUT, waits
 // (bounded) for what it issued, frees TMEM and returns.
@@ -376,9 +379,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_consta
           m_ref = mx;
         }
         // P = exp2(s * c2 - m_ref) in bf16 over the tile's S columns (keys 2c, 2c + 1 in
-        // column c), the argument two at a time in one packed fma, a quarter of the pairs'
-        // exponentials on the FMA pipe; l sums the bf16 values the MMA consumes, two at a time
-        // in packed adds
+        // column c), the argument two at a time in one packed fma, one pair in eight on the
+        // FMA pipe; l sums the bf16 values the MMA consumes, two at a time in packed adds
         const float2 c2x2 = make_float2(a.c2, a.c2), nm = make_float2(-m_ref, -m_ref);
         float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
