@@ -705,8 +705,9 @@ bool expand_tc_supported(const mla_config& c) {
          (c.num_heads * c.head_dim) % 128 == 0 && (c.num_heads * c.head_dim_v) % 128 == 0;
 }
 
-// Workspace: Q (n, H, d_h + d_r), K_nope (n, H * d_h), V (n, H * d_v) in dtype, then the
-// expansion's partial sums.
+// Workspace: the query (n, H, d_r) rotated for the tensor cores, else (n, H, d_h + d_r)
+// packed; K_nope (n, H * d_h), V (n, H * d_v) in dtype; then the front end's partial sums
+// where its weight stream does the expansion.
 struct PrefillLayout {
   size_t q, kn, v, part, total;
 };
@@ -716,11 +717,16 @@ PrefillLayout prefill_layout(const mla_config& c, int n) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   PrefillLayout L;
   L.q = 0;
-  L.kn = up((size_t)n * c.num_heads * (c.head_dim + c.rope_dim) * e);
+  // the tensor-core attention takes only the rotated RoPE part of the query from here
+  const int qd = prefill_tc_supported(c) ? c.rope_dim : c.head_dim + c.rope_dim;
+  L.kn = up((size_t)n * c.num_heads * qd * e);
   L.v = L.kn + up((size_t)n * c.num_heads * c.head_dim * e);
   L.part = L.v + up((size_t)n * c.num_heads * c.head_dim_v * e);
+  // partial sums only for the front end's weight stream (the expansion GEMM writes K and V)
   const int rows[2] = {c.num_heads * c.head_dim, c.num_heads * c.head_dim_v};
-  L.total = L.part + up(front_part_bytes(c, c.kv_rank, n, rows, 2, false));
+  L.total = L.part + (expand_tc_supported(c)
+                          ? 0
+                          : up(front_part_bytes(c, c.kv_rank, n, rows, 2, false)));
   return L;
 }
 
