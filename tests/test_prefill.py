@@ -64,6 +64,25 @@ def test_prefill_validates_arguments(mla):
     assert call(q) == mla.MLA_ERR_INVALID_ARG
 
 
+def test_prefill_workspace_layout(mla):
+    """The tensor-core path's workspace is the rotated RoPE query, K_nope and V in bf16 (80 KB
+    per token at the DeepSeek-V2 heads), each region 256-byte aligned; the CUDA-core path
+    also holds the packed query and the front end's partial sums."""
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    w = mi.WORKLOADS["dsv2"]
+    c = _cfg(mla, w).c()
+    H, dh, dr, dv = w.num_heads, w.head_dim, w.rope_dim, w.head_dim_v
+    for n in (1, 7, 1000, 16384):
+        want = up(n * H * dr * 2) + up(n * H * dh * 2) + up(n * H * dv * 2)
+        assert mla.lib.mla_prefill_workspace_size(ctypes.byref(c), n) == want, n
+    assert mla.lib.mla_prefill_workspace_size(ctypes.byref(c), 16384) == 1280 * 2 ** 20
+    w = mi.WORKLOADS["small_fp32"]
+    c = _cfg(mla, w).c()
+    H, dh, dr, dv = w.num_heads, w.head_dim, w.rope_dim, w.head_dim_v
+    n = 1000
+    assert mla.lib.mla_prefill_workspace_size(ctypes.byref(c), n) >= n * H * (dh + dr + dh + dv) * 4
+
+
 def _run(mla, w, lens, seed=5, sample=None):
     """Device prefill of sequences of the given lengths, and the oracle's outputs (for the
     query tokens sample[b] of sequence b when a sample is given, else for every token)."""
